@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer hot path (route -> dispatch -> grouped FFN ->
+combine) on B200, printing one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode]
+  python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+One step = one whole layer over one batch of the workload (default: the
+decode layer, T=128, H=7168, E=256, top-8, I=2048, FP8 block-scaled weights).
+Under torchrun every rank runs its own replica on its own GPU (the layer has no
+data-path collective); value = tokens of all ranks / max over ranks of the
+device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer µs & tokens/s (decode T=128, prefill T=8192); % of HBM/FP8 roofline"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="decode")
+    p.add_argument("--T", type=int, default=None, help="override the token count")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="wall-clock budget of the CPU oracle sample")
+    return p.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), \
+        int(os.environ.get("WORLD_SIZE", 1))
+
+
+# ------------------------------------------------------------ GPU clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3][1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None):
+    """Time the CPU oracle on the first tokens of the workload until `seconds`
+    of wall time are spent. Returns (tokens, elapsed_s, cores)."""
+    import numpy as np
+    import torch
+    import oracle
+
+    cores = len(os.sched_getaffinity(0))
+    odt = {"f32": oracle.F32, "bf16": oracle.BF16, "e4m3": oracle.E4M3}
+
+    def host(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    logits = host(inp["logits"])
+    x = host(inp["x"])
+    idx, _ = oracle.route(logits, spec.k, spec.renorm)
+    limit = spec.T if max_tokens is None else min(spec.T, max_tokens)
+    chunk = max(1, min(cores, limit))
+    done = 0
+    elapsed = 0.0
+    while done < limit and elapsed < seconds:
+        t1 = min(limit, done + chunk)
+        kw = {}
+        if not spec.identity:
+            experts = sorted(set(idx[done:t1].ravel().tolist()))
+            for n in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
+                if inp.get(n) is not None:
+                    kw[n] = {e: host(inp[n][e]) for e in experts}
+        p = oracle.Problem(spec.T, spec.H, spec.E, spec.k, spec.I, x_dtype=odt[spec.act],
+                           xq_dtype=odt[spec.xq], w_dtype=odt[spec.weight], h_dtype=odt[spec.h],
+                           y_dtype=odt[spec.y], out_dtype=odt[spec.out], renorm=spec.renorm,
+                           identity=spec.identity, **kw)
+        t_start = time.perf_counter()
+        oracle.moe_layer(p, x, logits, done, t1)
+        elapsed += time.perf_counter() - t_start
+        done = t1
+    return done, elapsed, cores
+
+
+# ------------------------------------------------------------ roofline --
+
+def ffn_algorithmic_bytes(spec, counts):
+    """Bytes the grouped FFN must move at least once: the weights of every
+    touched expert (matrices + scales), the dispatched rows read, h written
+    and read back, y written."""
+    from combine_softmax_top_b200 import workloads as W
+    el = {"f32": 4, "bf16": 2, "e4m3": 1}
+    touched = int((counts > 0).sum())
+    rows = int(counts.sum())
+    w = touched * W.bytes_per_expert(spec)
+    xs = spec.H // 128 * 4 if spec.xq == "e4m3" else 0
+    hs = spec.I // 128 * 4 if spec.h == "e4m3" else 0
+    act = rows * (spec.H * el[spec.xq] + xs) + 2 * rows * (spec.I * el[spec.h] + hs) \
+        + rows * spec.H * el[spec.y]
+    return w + act, touched
+
+
+def ffn_flops(spec, rows):
+    return 6.0 * spec.H * spec.I * rows
+
+
+def recorded_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel (else None)."""
+    path = os.path.join(PROFILES, "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel_tag)
+    if not rec:
+        return None
+    if rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_softmax_top_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("ffn_") or name.endswith(".cuh"):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------ reference --
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    from combine_softmax_top_b200 import workloads as W
+    import torch
+    spec = W.spec(args.config, **({"T": args.T} if args.T else {}))
+    inp = W.make_inputs(spec, seed=args.seed, device="cpu")
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(spec, inp, per_step / 4)
+    tok = el = 0.0
+    cores = 1
+    for _ in range(args.steps):
+        n, e, cores = oracle_sample(spec, inp, per_step)
+        tok += n
+        el += e
+    value = tok / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * spec.T / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
+        "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
+                               f"top-{spec.k} I={spec.I}", "T": spec.T},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first tokens of each step until {per_step:.1f}s of CPU wall time"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------ ours --
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from combine_softmax_top_b200 import moe
+    from combine_softmax_top_b200 import workloads as W
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    spec = W.spec(args.config, **({"T": args.T} if args.T else {}))
+    inp = W.make_inputs(spec, seed=args.seed + rank, device=dev)
+    b = moe.alloc_buffers(spec, device=dev)
+    w = moe.weights_struct(inp) if not spec.identity else moe.moe_weights()
+    bufs = b.dispatch_bufs()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws, stream)
+        if ev:
+            ev[1].record(stream)
+        moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, bufs, stream)
+        if ev:
+            ev[2].record(stream)
+        if not spec.identity:
+            moe.moe_grouped_ffn(b.shape, bufs, w, b.ws, b.y, stream)
+        if ev:
+            ev[3].record(stream)
+        moe.moe_combine(b.shape, bufs, b.y, b.topk_w, b.ws, b.out, stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    rc = moe.moe_poll_status(b.ws, stream)
+    if rc != 0:
+        raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for i in range(args.steps):
+        flush.zero_()                      # L2 flushed between timed steps
+        step(evs[i])
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    rc = moe.moe_poll_status(b.ws, stream)
+    if rc != 0:
+        raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
+
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                      for i in range(args.steps)])          # ms
+    step_ms = stage.sum(1)
+    my_ms = float(step_ms.mean())
+    if world > 1:
+        t = torch.tensor([my_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    else:
+        ms = my_ms
+    tokens_all = spec.T * world
+    value = tokens_all / (ms / 1000.0)
+
+    # end to end through the C ABI with host buffers: H2D of x and logits,
+    # the layer, D2H of the output, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = inp["x"].cpu().pin_memory()
+        hl = inp["logits"].cpu().pin_memory()
+        ho = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+        dx = torch.empty_like(inp["x"])
+        dl = torch.empty_like(inp["logits"])
+        e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for i in range(args.steps + 2):
+            flush.zero_()
+            if i >= 2:
+                e_evs[i - 2][0].record(stream)
+            dx.copy_(hx, non_blocking=True)
+            dl.copy_(hl, non_blocking=True)
+            moe.moe_layer(b.shape, dx, dl, w, b.topk_idx, b.topk_w, bufs, b.y, b.ws, b.out, stream)
+            ho.copy_(b.out, non_blocking=True)
+            if i >= 2:
+                e_evs[i - 2][1].record(stream)
+        torch.cuda.synchronize()
+        e_ms = statistics.mean(a.elapsed_time(z) for a, z in e_evs)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": tokens_all / (e_ms / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": hx.numel() * hx.element_size() + hl.numel() * hl.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+
+    counts = b.counts.cpu().numpy()
+    peaks, peak_kind = load_peaks()
+    ffn_ms = float(stage[:, 2].mean())
+    roofline = None
+    if not spec.identity:
+        abytes, touched = ffn_algorithmic_bytes(spec, counts)
+        flops = ffn_flops(spec, int(counts.sum()))
+        bw = abytes / (ffn_ms / 1000.0) / 1e9
+        # decode-size GEMMs stream weights (HBM bound); big-batch GEMMs are
+        # bound by the tensor pipe
+        t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12 * (2.0 if spec.weight == "e4m3" else 1.0))
+        if t_hbm >= t_tc:
+            roofline = {"bound": "hbm", "achieved": bw, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": bw / peaks["hbm_gbs"]}
+        else:
+            pk = peaks["bf16_tflops"] * (2.0 if spec.weight == "e4m3" else 1.0)
+            ach = flops / (ffn_ms / 1000.0) / 1e12
+            roofline = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                        "frac": ach / pk}
+        roofline.update({"kernel": "grouped_ffn", "algorithmic_bytes_per_launch": abytes,
+                         "flops_per_launch": flops, "touched_experts": touched,
+                         "launch_ms": ffn_ms, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback",
+                         "traffic": recorded_traffic(f"grouped_ffn/{spec.name}")})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, el, cores = oracle_sample(spec, inp, args.cpu_seconds)
+        cpu = {"value": n / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n} of {spec.T} tokens of the same workload ({el:.1f}s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "us_per_layer": ms * 1000.0, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3" if spec.weight == "e4m3" else spec.weight,
+            "data": "synthetic (seeded; random-init weights, no checkpoint)",
+            "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
+                                   f"top-{spec.k} I={spec.I} "
+                                   f"{'e4m3 128x128-block weights, bf16 tokens' if spec.weight == 'e4m3' else spec.weight}",
+                       "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MB write) before every timed step; weights 11 GB > L2"},
+            "stage_us": {k: float(stage[:, j].mean() * 1000.0)
+                         for j, k in enumerate(["route", "dispatch", "grouped_ffn", "combine"])},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * moe.kernels_per_layer(spec),
+            "clocks": clk,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

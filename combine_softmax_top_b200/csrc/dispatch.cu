@@ -1,0 +1,254 @@
+// One-pass dispatch into expert-major windows.
+//
+// Pages: tokens are pushed straight into the destination windows without a
+// metadata exchange first, and the grouped GEMM reads them there in place
+// (NVLinkOneSided abstract); a ready flag travels with the data (its
+// "Sentinel" protocol); the producer bumps a counter per batch of filled ring
+// blocks that the GEMM polls, and double-buffered counters remove the clean
+// pass between calls (GC-MoE explainer, "Three-Node CUDA Graph and token-ring
+// Handshake"). Only counts, offsets and sync metadata are kept (Ascend report,
+// abstract).
+//
+// One CTA per token:
+//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j;
+//  2. all warps stream the token row once (16-byte loads) and write it to the
+//     k claimed rows; E4M3 rows are quantised per 128 values with the
+//     smallest power-of-two scale that keeps the block within +-448, and the
+//     scale's exponent byte also goes to the tile's scale-factor atom read by
+//     the block-scaled MMA;
+//  3. each slot bumps its tile's fill counter; the bump that completes 128 rows
+//     publishes the tile (sentinel + ring entry);
+//  4. the CTA that finishes the last token closes: it publishes the partial
+//     last tile of each expert, writes counts/offsets and the tile total, and
+//     advances the epoch.
+// Every CTA first zeroes its share of the counter set the *next* dispatch will
+// use, so no separate clean pass is needed.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kElems = 16;  // values per lane per step
+
+struct Args {
+  const void* x;
+  const int32_t* idx;
+  int T, H, E, k, cap, tpe;
+  int act, xq_dtype;
+  moe_dispatch_bufs b;
+  Ws ws;
+  int64_t set_words;
+};
+
+__device__ __forceinline__ void load16(const void* x, int act, int64_t off, float* v) {
+  if (act == MOE_BF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + off);
+    uint4 a = __ldg(p), b = __ldg(p + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 q = __ldg(p + i);
+      v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+    }
+  }
+}
+
+__device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e, int tile,
+                             int rows) {
+  st_release(a.ws.sentinel + (int64_t)e * a.tpe + tile, (epoch << 8) | (uint32_t)rows);
+  const uint32_t slot = atomicAdd(set + a.E + a.E * a.tpe + kRingHead, 1u);
+  st_release64(a.ws.ring + slot,
+               ((unsigned long long)epoch << 32) | ((unsigned long long)e << 16) | (unsigned)tile);
+}
+
+__global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
+  __shared__ int s_row[kMaxTopk];
+  __shared__ int s_e[kMaxTopk];
+  __shared__ uint32_t s_epoch;
+  __shared__ int s_last;
+  __shared__ uint32_t s_tiles;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_epoch = a.ws.hdr->epoch_next;
+  __syncthreads();
+  const uint32_t epoch = s_epoch;
+  uint32_t* set = a.ws.set[epoch & 1];
+  uint32_t* next = a.ws.set[(epoch + 1) & 1];
+  uint32_t* count = set;
+  uint32_t* fill = set + a.E;
+  uint32_t* misc = set + a.E + (int64_t)a.E * a.tpe;
+
+  // zero this CTA's share of the next counter set
+  {
+    const int64_t per = (a.set_words + gridDim.x - 1) / gridDim.x;
+    const int64_t lo = per * blockIdx.x;
+    const int64_t hi = min(lo + per, a.set_words);
+    for (int64_t i = lo + tid; i < hi; i += kThreads) next[i] = 0u;
+  }
+
+  const int t = blockIdx.x;
+  if (t < a.T) {
+    // 1. claim rows
+    if (tid < a.k) {
+      const int pair = t * a.k + tid;
+      const int e = __ldg(a.idx + pair);
+      int row = -1;
+      if (e >= 0 && e < a.E) {
+        const uint32_t p = atomicAdd(count + e, 1u);
+        if (p < (uint32_t)a.cap) {
+          row = e * a.cap + (int)p;
+          a.b.row_src[row] = pair;
+        } else {
+          latch_error(a.ws.hdr, MOE_ERR_CAPACITY, (uint32_t)e);
+        }
+      } else {
+        latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, (uint32_t)pair);
+      }
+      a.b.pos[pair] = row;
+      s_row[tid] = row;
+      s_e[tid] = e;
+    }
+    __syncthreads();
+
+    // 2. stream the row: lane group of 8 covers one 128-value block
+    const int steps = a.H / kElems;
+    for (int s = tid; s < (steps + 31) / 32 * 32; s += kThreads) {
+      const bool live = s < steps;
+      const int h0 = s * kElems;
+      float v[kElems];
+      if (live) load16(a.x, a.act, (int64_t)t * a.H + h0, v);
+      else {
+#pragma unroll
+        for (int i = 0; i < kElems; ++i) v[i] = 0.f;
+      }
+      if (a.xq_dtype == MOE_E4M3) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < kElems; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        if (!live) continue;
+        const int p = pow2_scale_exp(amax);
+        const float inv = exp2i(-p > -126 ? -p : -126);  // 2^-p; p <= 120 for finite x
+        uint32_t q[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint16_t lo = cvt_e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv);
+          uint16_t hi = cvt_e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+          q[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+        const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+        const bool leader = (tid & 7) == 0;
+        const int blk = h0 / kQBlock;
+        for (int j = 0; j < a.k; ++j) {
+          const int row = s_row[j];
+          if (row < 0) continue;
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
+          if (leader) {
+            a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
+            const int tile = row / kTileRows;   // global tile id e * tpe + local (cap % 128 == 0)
+            const int m = row % kTileRows;
+            a.ws.xsf[((int64_t)tile * ((a.H + 511) / 512) + blk / 4) * kSfAtomBytes +
+                     sf_atom_offset(m, blk & 3)] = (uint8_t)(p + 127);
+          }
+        }
+      } else if (live) {
+        for (int j = 0; j < a.k; ++j) {
+          const int row = s_row[j];
+          if (row < 0) continue;
+          const int64_t off = (int64_t)row * a.H + h0;
+          if (a.xq_dtype == MOE_BF16) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+              w[i] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.b.xq) + off);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.b.xq) + off);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+      }
+    }
+    __threadfence();
+    __syncthreads();
+
+    // 3. count the filled rows; the bump that completes a tile publishes it
+    if (tid < a.k) {
+      const int row = s_row[tid];
+      if (row >= 0) {
+        const int e = s_e[tid];
+        const int local = row - e * a.cap;
+        const int tile = local / kTileRows;
+        const uint32_t old = atomicAdd(fill + (int64_t)e * a.tpe + tile, 1u);
+        if (old + 1 == (uint32_t)kTileRows) publish_tile(a, set, epoch, e, tile, kTileRows);
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+
+  // 4. the last CTA closes
+  if (tid == 0) s_last = atomicAdd(misc + kDone, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (tid == 0) s_tiles = 0;
+  __syncthreads();
+  for (int e = tid; e < a.E; e += kThreads) {
+    const uint32_t c_raw = ld_acquire(count + e);
+    const int c = (int)min(c_raw, (uint32_t)a.cap);
+    a.b.counts[e] = c;
+    a.b.offsets[e] = e * a.cap;
+    const int full = c / kTileRows;
+    const int rem = c % kTileRows;
+    if (rem) publish_tile(a, set, epoch, e, full, rem);   // the partial last tile
+    atomicAdd(&s_tiles, (uint32_t)(full + (rem ? 1 : 0)));
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    st_release(misc + kRingTotal, s_tiles);
+    a.ws.hdr->epoch_cur = epoch;
+    __threadfence();
+    a.ws.hdr->epoch_next = epoch + 1;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
+                            const moe_dispatch_bufs& b) {
+  Args a;
+  a.x = x;
+  a.idx = idx;
+  a.T = (int)c.s.T;
+  a.H = (int)c.s.H;
+  a.E = (int)c.s.E;
+  a.k = (int)c.s.topk;
+  a.cap = (int)c.L.cap;
+  a.tpe = (int)c.L.tpe;
+  a.act = c.s.act_dtype;
+  a.xq_dtype = c.s.xq_dtype;
+  a.b = b;
+  a.ws = c.ws;
+  a.set_words = (int64_t)c.L.set_words;
+  const int grid = a.T > 0 ? a.T : 1;
+  dispatch_kernel<<<grid, kThreads, 0, c.stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

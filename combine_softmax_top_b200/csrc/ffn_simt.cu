@@ -1,0 +1,232 @@
+// Grouped expert FFN on the CUDA cores (fp32 FFMA), for the fp32 layer.
+//
+// Same schedule as the tensor-core kernel, without tensor cores: work units
+// are (published tile, 128-feature slice); each unit waits for its tile's
+// sentinel, then computes G and U (gate/up pass) or y (down pass) for up to
+// 128 rows in 32-row steps with shared-memory tiles of 32 along K.
+// h = silu(G) * U (SwiGLU, GC-MoE feed item "Full text"), requantised per 128
+// values when stored as e4m3.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kF = 128;   // features per unit
+constexpr int kR = 32;    // rows per step
+constexpr int kK = 32;    // K per shared-memory stage
+
+struct Args {
+  const void* xq;  const float* xs;     // gate/up input rows
+  void* hq;        float* hs;           // SwiGLU output rows
+  void* y;
+  const void* wg;  const void* wu;  const void* wd;
+  const float* sg; const float* su; const float* sd;
+  int H, I, E, cap, tpe;
+  int xq_dt, w_dt, h_dt, y_dt;
+  Ws ws;
+  uint8_t* hsf;
+  int64_t igroups;
+};
+
+__device__ __forceinline__ float ld_act(const void* p, int dt, int64_t i) {
+  if (dt == MOE_F32) return reinterpret_cast<const float*>(p)[i];
+  if (dt == MOE_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return e4m3_to_f32(reinterpret_cast<const uint8_t*>(p)[i]);
+}
+
+// Find the tile behind ring slot `slot` for the current epoch (bounded wait).
+__device__ bool fetch_tile(const Args& a, uint32_t epoch, uint32_t slot, int* e, int* tile,
+                           int* rows) {
+  const unsigned long long t0 = globaltimer();
+  unsigned long long ent;
+  while (true) {
+    ent = ld_acquire64(a.ws.ring + slot);
+    if ((uint32_t)(ent >> 32) == epoch) break;
+    if (globaltimer() - t0 > kWaitBudgetNs) {
+      latch_error(a.ws.hdr, MOE_ERR_TIMEOUT, slot);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  *e = (int)((ent >> 16) & 0xFFFF);
+  *tile = (int)(ent & 0xFFFF);
+  const uint32_t* sp = a.ws.sentinel + (int64_t)(*e) * a.tpe + *tile;
+  while (true) {
+    const uint32_t s = ld_acquire(sp);
+    if ((s >> 8) == (epoch & 0xFFFFFFu)) { *rows = (int)(s & 0xFF); return true; }
+    if (globaltimer() - t0 > kWaitBudgetNs) {
+      latch_error(a.ws.hdr, MOE_ERR_TIMEOUT, slot);
+      return false;
+    }
+    __nanosleep(256);
+  }
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.f + expf(-g)); }
+
+// DOWN = false: gate/up + SwiGLU; DOWN = true: y = h W_down^T
+template <bool DOWN>
+__global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
+  __shared__ float sx[kR][kK + 1];
+  __shared__ float sw0[kF][kK + 1];
+  __shared__ float sw1[DOWN ? 1 : kF][kK + 1];
+  __shared__ float samax[kR][4];
+  __shared__ int s_info[4];
+
+  const int tid = threadIdx.x;
+  const int f = tid & (kF - 1);
+  const int rh = tid >> 7;          // rows rh*16 .. rh*16+15 of a step
+  const int K = DOWN ? a.I : a.H;
+  const int NF = DOWN ? a.H : a.I;  // output features
+  const int nslices = NF / kF;
+  const uint32_t epoch = a.ws.hdr->epoch_cur;
+  const uint32_t* misc = a.ws.set[epoch & 1] + a.E + (int64_t)a.E * a.tpe;
+  const uint32_t total = ld_acquire(misc + kRingTotal);
+  const void* xin = DOWN ? a.hq : a.xq;
+  const float* xsc = DOWN ? a.hs : a.xs;
+  const int xdt = DOWN ? a.h_dt : a.xq_dt;
+
+  for (uint32_t u = blockIdx.x; u < total * (uint32_t)nslices; u += gridDim.x) {
+    const uint32_t slot = u / nslices;
+    const int slice = (int)(u % nslices);
+    if (tid == 0) {
+      int e = 0, tile = 0, rows = 0;
+      const bool ok = fetch_tile(a, epoch, slot, &e, &tile, &rows);
+      s_info[0] = ok ? e : -1; s_info[1] = tile; s_info[2] = rows;
+    }
+    __syncthreads();
+    const int e = s_info[0], tile = s_info[1], rows = s_info[2];
+    __syncthreads();
+    if (e < 0) continue;
+    const int64_t row0 = (int64_t)e * a.cap + (int64_t)tile * kTileRows;
+    const int f0 = slice * kF;
+    const void* w0 = DOWN ? a.wd : a.wg;
+    const void* w1 = a.wu;
+    const float* s0 = DOWN ? a.sd : a.sg;
+    const float* s1 = a.su;
+    const int64_t wrow0 = (int64_t)e * NF + f0;   // first weight row of this unit
+
+    for (int r0 = 0; r0 < rows; r0 += kR) {
+      float g[16], uu[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) { g[i] = 0.f; uu[i] = 0.f; }
+      for (int k0 = 0; k0 < K; k0 += kK) {
+        for (int i = tid; i < kR * kK; i += kThreads) {
+          const int r = i / kK, kk = i % kK;
+          float v = 0.f;
+          if (r0 + r < rows) {
+            const int64_t row = row0 + r0 + r;
+            v = ld_act(xin, xdt, row * K + k0 + kk);
+            if (xdt == MOE_E4M3) v *= xsc[row * (K / kQBlock) + (k0 + kk) / kQBlock];
+          }
+          sx[r][kk] = v;
+        }
+        float sc0 = 1.f, sc1 = 1.f;
+        if (a.w_dt == MOE_E4M3) {
+          const int64_t sidx = ((int64_t)e * (NF / kQBlock) + f0 / kQBlock) * (K / kQBlock) + k0 / kQBlock;
+          sc0 = s0[sidx];
+          if (!DOWN) sc1 = s1[sidx];
+        }
+        for (int i = tid; i < kF * kK; i += kThreads) {
+          const int ff = i / kK, kk = i % kK;
+          const int64_t widx = (wrow0 + ff) * K + k0 + kk;
+          sw0[ff][kk] = ld_act(w0, a.w_dt, widx) * sc0;
+          if (!DOWN) sw1[ff][kk] = ld_act(w1, a.w_dt, widx) * sc1;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < kK; ++kk) {
+          const float b0 = sw0[f][kk];
+          const float b1 = DOWN ? 0.f : sw1[f][kk];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float xv = sx[rh * 16 + i][kk];
+            g[i] = fmaf(xv, b0, g[i]);
+            if (!DOWN) uu[i] = fmaf(xv, b1, uu[i]);
+          }
+        }
+        __syncthreads();
+      }
+
+      if (DOWN) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = r0 + rh * 16 + i;
+          if (r >= rows) break;
+          const int64_t o = (row0 + r) * a.H + f0 + f;
+          if (a.y_dt == MOE_F32) reinterpret_cast<float*>(a.y)[o] = g[i];
+          else reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(g[i]);
+        }
+        continue;
+      }
+      float h[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h[i] = silu(g[i]) * uu[i];
+      if (a.h_dt == MOE_E4M3) {
+        const int warp = (tid >> 5) & 3;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float m = fabsf(h[i]);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          if ((tid & 31) == 0) samax[rh * 16 + i][warp] = m;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int rr = rh * 16 + i;
+          const int r = r0 + rr;
+          const float m = fmaxf(fmaxf(samax[rr][0], samax[rr][1]), fmaxf(samax[rr][2], samax[rr][3]));
+          const int p = pow2_scale_exp(m);
+          if (r < rows) {
+            const int64_t row = row0 + r;
+            const float q = h[i] * exp2i(-p > -126 ? -p : -126);
+            const uint16_t b2 = cvt_e4m3x2(q, 0.f);
+            reinterpret_cast<uint8_t*>(a.hq)[row * a.I + f0 + f] = (uint8_t)(b2 & 0xFF);
+            if (f == 0) {
+              a.hs[row * (a.I / kQBlock) + slice] = exp2i(p);
+              if (a.hsf)
+                a.hsf[((int64_t)(row / kTileRows) * a.igroups + slice / 4) * kSfAtomBytes +
+                      sf_atom_offset((int)(row % kTileRows), slice & 3)] = (uint8_t)(p + 127);
+            }
+          }
+        }
+        __syncthreads();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = r0 + rh * 16 + i;
+          if (r >= rows) break;
+          const int64_t o = (row0 + r) * a.I + f0 + f;
+          if (a.h_dt == MOE_F32) reinterpret_cast<float*>(a.hq)[o] = h[i];
+          else reinterpret_cast<__nv_bfloat16*>(a.hq)[o] = __float2bfloat16_rn(h[i]);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,
+                            void* y) {
+  Args a;
+  a.xq = b.xq; a.xs = b.xs; a.hq = b.hq; a.hs = b.hs; a.y = y;
+  a.wg = w.w_gate; a.wu = w.w_up; a.wd = w.w_down;
+  a.sg = w.s_gate; a.su = w.s_up; a.sd = w.s_down;
+  a.H = (int)c.s.H; a.I = (int)c.s.I; a.E = (int)c.s.E;
+  a.cap = (int)c.L.cap; a.tpe = (int)c.L.tpe;
+  a.xq_dt = c.s.xq_dtype; a.w_dt = c.s.weight_dtype; a.h_dt = c.s.h_dtype; a.y_dt = c.s.y_dtype;
+  a.ws = c.ws;
+  a.hsf = c.s.h_dtype == MOE_E4M3 ? c.ws.hsf : nullptr;
+  a.igroups = c.L.igroups;
+  const int grid = c.num_sms * 4;
+  ffn_simt_kernel<false><<<grid, kThreads, 0, c.stream>>>(a);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ffn_simt_kernel<true><<<grid, kThreads, 0, c.stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

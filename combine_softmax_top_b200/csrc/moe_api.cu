@@ -1,0 +1,229 @@
+// Host side of the C ABI declared in include/moe.h: argument checks, the
+// workspace, and the kernel launches of each stage.
+#include <cstring>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool is_dtype(int32_t d) { return d == MOE_F32 || d == MOE_BF16 || d == MOE_E4M3; }
+
+// Shape and dtype checks shared by every entry point.
+moe_status check_shape(const moe_shape* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->E < 1 || s->E > 65535) return MOE_ERR_INVALID_ARG;
+  if (s->topk < 1 || s->topk > s->E || s->topk > kMaxTopk) return MOE_ERR_INVALID_ARG;
+  if (s->quant_block != kQBlock || s->flags != 0) return MOE_ERR_INVALID_ARG;
+  if ((s->renorm != 0 && s->renorm != 1) || (s->identity_experts != 0 && s->identity_experts != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (s->cap_rows < 0 || (s->cap_rows > 0 && s->cap_rows % kTileRows != 0)) return MOE_ERR_INVALID_ARG;
+  if (s->E > 1024) return MOE_ERR_UNSUPPORTED;      // route keeps a row in registers
+  if (s->H % 16 != 0 || s->H > (1 << 24)) return MOE_ERR_INVALID_ARG;
+  if (!is_dtype(s->act_dtype) || !is_dtype(s->xq_dtype) || !is_dtype(s->out_dtype))
+    return MOE_ERR_INVALID_ARG;
+  if (s->act_dtype == MOE_E4M3 || s->out_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (s->xq_dtype == MOE_E4M3 && s->H % kQBlock != 0) return MOE_ERR_INVALID_ARG;
+  const int64_t cap = default_cap(*s);
+  if (cap / kTileRows > 65535 || s->E * cap >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (s->T * s->topk >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (s->identity_experts) return MOE_OK;
+  if (s->I <= 0 || s->I > (1 << 24) || s->I % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (!is_dtype(s->weight_dtype) || !is_dtype(s->h_dtype) || !is_dtype(s->y_dtype))
+    return MOE_ERR_INVALID_ARG;
+  if (s->y_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  const bool f32 = s->act_dtype == MOE_F32 && s->xq_dtype == MOE_F32 && s->weight_dtype == MOE_F32 &&
+                   s->h_dtype == MOE_F32 && s->y_dtype == MOE_F32 && s->out_dtype == MOE_F32;
+  const bool bf16 = s->act_dtype == MOE_BF16 && s->xq_dtype == MOE_BF16 &&
+                    s->weight_dtype == MOE_BF16 && s->h_dtype == MOE_BF16 &&
+                    s->y_dtype == MOE_BF16 && s->out_dtype == MOE_BF16;
+  const bool fp8 = s->act_dtype == MOE_BF16 && s->xq_dtype == MOE_E4M3 &&
+                   s->weight_dtype == MOE_E4M3 && s->h_dtype == MOE_E4M3 &&
+                   s->y_dtype == MOE_BF16 && s->out_dtype == MOE_BF16;
+  if (!f32 && !bf16 && !fp8) return MOE_ERR_UNSUPPORTED;
+  // the expert FFN kernels work on 128-feature slices
+  if (s->H % kQBlock != 0 || s->I % kQBlock != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status make_ctx(const moe_shape* s, void* ws, moe_stream_t stream, Ctx* c) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!ws || ((uintptr_t)ws & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  c->s = *s;
+  c->L = make_layout(*s);
+  c->ws = ws_view(ws, c->L);
+  c->stream = (cudaStream_t)stream;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_h) {
+  if (!b) return MOE_ERR_INVALID_ARG;
+  if (!b->xq || !b->counts || !b->offsets || !b->row_src || !b->pos) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(b->xq)) return MOE_ERR_INVALID_ARG;
+  if (s->xq_dtype == MOE_E4M3 && (!b->xs || !aligned16(b->xs))) return MOE_ERR_INVALID_ARG;
+  if (need_h && !s->identity_experts) {
+    if (!b->hq || !aligned16(b->hq)) return MOE_ERR_INVALID_ARG;
+    if (s->h_dtype == MOE_E4M3 && (!b->hs || !aligned16(b->hs))) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_shape* s, const moe_weights* w) {
+  if (!w || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
+  if (s->weight_dtype == MOE_E4M3 && (!w->s_gate || !w->s_up || !w->s_down)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+__global__ void init_ws_kernel(uint32_t* words, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    words[i] = 0u;
+  if (blockIdx.x == 0 && threadIdx.x == 0) words[0] = 1u;   // Header::epoch_next
+}
+
+moe_status do_route(const Ctx& c, const float* logits, int32_t* idx, float* w) {
+  if (!logits || !idx || !w || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route(c, logits, idx, w));
+}
+
+moe_status do_dispatch(const Ctx& c, const void* x, const int32_t* idx, const moe_dispatch_bufs* b) {
+  if (!x || !idx || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_bufs(&c.s, b, false);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_dispatch(c, x, idx, *b));
+}
+
+moe_status do_ffn(const Ctx& c, const moe_dispatch_bufs* b, const moe_weights* w, void* y) {
+  if (c.s.identity_experts) return MOE_OK;
+  moe_status st = check_bufs(&c.s, b, true);
+  if (st != MOE_OK) return st;
+  st = check_weights(&c.s, w);
+  if (st != MOE_OK) return st;
+  if (!y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (ffn_tc_supported(c.s)) return cuda_status(launch_ffn_tc(c, *b, *w, y));
+  return cuda_status(launch_ffn_simt(c, *b, *w, y));
+}
+
+moe_status do_combine(const Ctx& c, const moe_dispatch_bufs* b, const void* y, const float* topk_w,
+                      void* out) {
+  if (!b || !b->pos || !topk_w || !out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (c.s.identity_experts) {
+    if (!b->xq || !aligned16(b->xq)) return MOE_ERR_INVALID_ARG;
+    if (c.s.xq_dtype == MOE_E4M3 && !b->xs) return MOE_ERR_INVALID_ARG;
+  } else if (!y || !aligned16(y)) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  return cuda_status(launch_combine(c, *b, y, topk_w, out));
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_bytes(const moe_shape* shape, size_t* bytes) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(*shape).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(const moe_shape* shape, void* ws, size_t bytes, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  if (st != MOE_OK) return st;
+  if (bytes < c.L.total) return MOE_ERR_INVALID_ARG;
+  // header, both counter sets, sentinels and ring (everything before the scale atoms)
+  const size_t words = c.L.off_xsf / 4;
+  const int grid = (int)std::min<size_t>((words + 255) / 256, (size_t)c.num_sms * 8);
+  init_ws_kernel<<<grid > 0 ? grid : 1, 256, 0, c.stream>>>((uint32_t*)ws, words);
+  return cuda_status(cudaGetLastError());
+}
+
+moe_status moe_route(const moe_shape* shape, const float* logits, int32_t* topk_idx, float* topk_w,
+                     void* ws, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  return st != MOE_OK ? st : do_route(c, logits, topk_idx, topk_w);
+}
+
+moe_status moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx, void* ws,
+                        const moe_dispatch_bufs* bufs, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  return st != MOE_OK ? st : do_dispatch(c, x, topk_idx, bufs);
+}
+
+moe_status moe_grouped_ffn(const moe_shape* shape, const moe_dispatch_bufs* bufs, const moe_weights* w,
+                           void* ws, void* y, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  return st != MOE_OK ? st : do_ffn(c, bufs, w, y);
+}
+
+moe_status moe_combine(const moe_shape* shape, const moe_dispatch_bufs* bufs, const void* y,
+                       const float* topk_w, void* ws, void* out, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  return st != MOE_OK ? st : do_combine(c, bufs, y, topk_w, out);
+}
+
+moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,
+                     int32_t* topk_idx, float* topk_w, const moe_dispatch_bufs* bufs, void* y,
+                     void* ws, void* out, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  if (st != MOE_OK) return st;
+  // every argument is checked before the first launch
+  if (!logits || !topk_idx || !topk_w || !aligned16(logits) || !x || !aligned16(x) || !out ||
+      !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  st = check_bufs(shape, bufs, true);
+  if (st != MOE_OK) return st;
+  if (!shape->identity_experts) {
+    st = check_weights(shape, w);
+    if (st != MOE_OK) return st;
+    if (!y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  }
+  if ((st = do_route(c, logits, topk_idx, topk_w)) != MOE_OK) return st;
+  if ((st = do_dispatch(c, x, topk_idx, bufs)) != MOE_OK) return st;
+  if ((st = do_ffn(c, bufs, w, y)) != MOE_OK) return st;
+  return do_combine(c, bufs, y, topk_w, out);
+}
+
+moe_status moe_poll_status(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t err = 0;
+  Header* h = (Header*)ws;
+  if (cudaMemcpy(&err, &h->error, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (err != 0 && cudaMemset(&h->error, 0, 8) != cudaSuccess) return MOE_ERR_CUDA;
+  return (moe_status)err;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype combination";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_CAPACITY: return "an expert received more rows than cap_rows";
+    case MOE_ERR_TIMEOUT: return "a device wait ran out of time";
+    case MOE_ERR_NONFINITE: return "non-finite router logits";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+// Internal definitions shared by the kernels and the host ABI of libmoe.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kTileRows = 128;   // rows per expert-window tile (sentinel granularity)
+constexpr int kQBlock = 128;     // quantisation block along H or I
+constexpr int kSfAtomBytes = 512;  // one scale-factor atom: 128 rows x 4 blocks
+constexpr int kMaxTopk = 32;
+
+// Waits give up after this long (ns of %globaltimer) and latch MOE_ERR_TIMEOUT.
+constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
+
+// ---- workspace layout -------------------------------------------------------
+//
+// [header 256 B][counter set 0][counter set 1][sentinels][ring][xsf][hsf]
+//
+// header : epoch_next, epoch_cur, error, error_info (u32 each)
+// set    : count[E] | fill[E*tpe] | misc[8] (ring_head, done, ring_total, ...)
+//          two sets are used alternately by consecutive dispatches; each
+//          dispatch zeroes the set the following dispatch will use.
+// sentinel[E*tpe] u32 : (epoch << 8) | rows of a published tile
+// ring[E*tpe] u64     : (epoch << 32) | (e << 16) | tile, in publication order
+// xsf / hsf           : UE8M0 scale atoms of xq / hq for the block-scaled MMA,
+//                       [tile][group of 4 blocks][512 B]
+struct Header {
+  uint32_t epoch_next;
+  uint32_t epoch_cur;
+  uint32_t error;
+  uint32_t error_info;
+  uint32_t pad[60];
+};
+static_assert(sizeof(Header) == 256, "header size");
+
+enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kMiscWords = 8 };
+
+struct Layout {
+  int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles = E * tpe
+  int64_t hgroups, igroups;                 // ceil(H/512), ceil(I/512)
+  size_t set_words;                         // u32 words of one counter set
+  size_t off_set[2], off_sentinel, off_ring, off_xsf, off_hsf, total;
+};
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+inline int64_t default_cap(const moe_shape& s) {
+  if (s.cap_rows > 0) return s.cap_rows;
+  int64_t c = ceil_div(s.T, kTileRows) * kTileRows;
+  return c < kTileRows ? kTileRows : c;
+}
+
+inline Layout make_layout(const moe_shape& s) {
+  Layout L{};
+  L.T = s.T; L.H = s.H; L.E = s.E; L.k = s.topk; L.I = s.I;
+  L.cap = default_cap(s);
+  L.tpe = ceil_div(L.cap, kTileRows);
+  L.tiles = L.E * L.tpe;
+  L.hgroups = ceil_div(L.H, 4 * kQBlock);
+  L.igroups = ceil_div(L.I, 4 * kQBlock);
+  L.set_words = (size_t)(L.E + L.tiles + kMiscWords);
+  size_t off = sizeof(Header);
+  for (int i = 0; i < 2; ++i) {
+    L.off_set[i] = off;
+    off = align_up(off + L.set_words * 4, 256);
+  }
+  L.off_sentinel = off;
+  off = align_up(off + (size_t)L.tiles * 4, 256);
+  L.off_ring = off;
+  off = align_up(off + (size_t)L.tiles * 8, 256);
+  L.off_xsf = off;
+  if (s.xq_dtype == MOE_E4M3) off = align_up(off + (size_t)L.tiles * L.hgroups * kSfAtomBytes, 256);
+  L.off_hsf = off;
+  if (s.h_dtype == MOE_E4M3 && !s.identity_experts)
+    off = align_up(off + (size_t)L.tiles * L.igroups * kSfAtomBytes, 256);
+  L.total = off;
+  return L;
+}
+
+// Device view of the workspace.
+struct Ws {
+  Header* hdr;
+  uint32_t* set[2];
+  uint32_t* sentinel;
+  unsigned long long* ring;
+  uint8_t* xsf;
+  uint8_t* hsf;
+};
+
+inline Ws ws_view(void* base, const Layout& L) {
+  char* b = (char*)base;
+  Ws w;
+  w.hdr = (Header*)b;
+  w.set[0] = (uint32_t*)(b + L.off_set[0]);
+  w.set[1] = (uint32_t*)(b + L.off_set[1]);
+  w.sentinel = (uint32_t*)(b + L.off_sentinel);
+  w.ring = (unsigned long long*)(b + L.off_ring);
+  w.xsf = (uint8_t*)(b + L.off_xsf);
+  w.hsf = (uint8_t*)(b + L.off_hsf);
+  return w;
+}
+
+// ---- device helpers -----------------------------------------------------------
+
+__device__ __forceinline__ void latch_error(Header* h, uint32_t code, uint32_t info) {
+  if (atomicCAS(&h->error, 0u, code) == 0u) atomicExch(&h->error_info, info);
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_release64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Exponent p of the smallest power of two 2^p >= amax / 448, clamped to
+// [-126, 127]; 0 for amax == 0. amax is a non-negative finite fp32 value.
+// 448 = 1.75 * 2^8: with amax = m * 2^e (m in [1, 2)), p = e - 8 when
+// m <= 1.75 and e - 7 otherwise. Exact integer work on the bit pattern.
+__device__ __forceinline__ int pow2_scale_exp(float amax) {
+  uint32_t b = __float_as_uint(amax);
+  if (b == 0u) return 0;
+  int e = (int)((b >> 23) & 0xFF);
+  if (e == 0) return -126;                      // subnormal amax
+  e -= 127;
+  int p = ((b & 0x7FFFFFu) > 0x600000u) ? e - 7 : e - 8;
+  return p < -126 ? -126 : (p > 127 ? 127 : p);
+}
+
+__device__ __forceinline__ float exp2i(int p) {  // 2^p for p in [-126, 127]
+  return __uint_as_float((uint32_t)(p + 127) << 23);
+}
+
+// Two fp32 values -> two e4m3 bytes (lo first in memory), nearest-even, satfinite.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  __nv_fp8x2_storage_t r = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+  return (uint16_t)r;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
+  __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q, __NV_E4M3);
+  return __half2float(__half(hr));
+}
+
+// Byte offset of (row m of a 128-row tile, block b of a 4-block group) inside
+// one scale-factor atom: 32 lanes x 16 bytes, lane m % 32, word m / 32, byte b.
+__device__ __forceinline__ int sf_atom_offset(int m, int b) {
+  return (m & 31) * 16 + (m >> 5) * 4 + b;
+}
+
+// ---- launchers (host, internal) --------------------------------------------
+
+struct Ctx {
+  moe_shape s;
+  Layout L;
+  Ws ws;
+  cudaStream_t stream;
+  int num_sms;
+};
+
+cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float* w);
+cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
+                            const moe_dispatch_bufs& b);
+cudaError_t launch_combine(const Ctx& c, const moe_dispatch_bufs& b, const void* y,
+                           const float* topk_w, void* out);
+cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,
+                            void* y);
+cudaError_t launch_ffn_tc(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,
+                          void* y);
+bool ffn_tc_supported(const moe_shape& s);
+
+}  // namespace moe

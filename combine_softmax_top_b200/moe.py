@@ -1,0 +1,257 @@
+"""Thin ctypes binding of libmoe.so (C ABI in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. torch supplies device memory and the current stream. If the library
+is missing or cannot be loaded the first call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from .workloads import BF16, E4M3, F32, Spec
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+_DT = {F32: MOE_F32, BF16: MOE_BF16, E4M3: MOE_E4M3}
+_TORCH = {F32: torch.float32, BF16: torch.bfloat16, E4M3: torch.uint8}
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+          4: "MOE_ERR_CAPACITY", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_NONFINITE"}
+
+EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
+           "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_poll_status", "moe_status_string")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("E", ctypes.c_int64),
+                ("topk", ctypes.c_int64), ("I", ctypes.c_int64),
+                ("act_dtype", ctypes.c_int32), ("xq_dtype", ctypes.c_int32),
+                ("weight_dtype", ctypes.c_int32), ("h_dtype", ctypes.c_int32),
+                ("y_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("renorm", ctypes.c_int32), ("identity_experts", ctypes.c_int32),
+                ("cap_rows", ctypes.c_int64), ("quant_block", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
+
+
+class moe_dispatch_bufs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("xq", "xs", "counts", "offsets", "row_src", "pos", "hq", "hs")]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it is absent: build it with
+    ``python -m combine_softmax_top_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m combine_softmax_top_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S = ctypes.c_void_p, ctypes.POINTER(moe_shape)
+        sig = {
+            "moe_workspace_bytes": [S, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_workspace_init": [S, P, ctypes.c_size_t, P],
+            "moe_route": [S, P, P, P, P, P],
+            "moe_dispatch": [S, P, P, P, ctypes.POINTER(moe_dispatch_bufs), P],
+            "moe_grouped_ffn": [S, ctypes.POINTER(moe_dispatch_bufs), ctypes.POINTER(moe_weights),
+                                P, P, P],
+            "moe_combine": [S, ctypes.POINTER(moe_dispatch_bufs), P, P, P, P, P],
+            "moe_layer": [S, P, P, ctypes.POINTER(moe_weights), P, P,
+                          ctypes.POINTER(moe_dispatch_bufs), P, P, P, P],
+            "moe_poll_status": [P, P],
+            "moe_status_string": [ctypes.c_int],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_char_p if name == "moe_status_string" else ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise MoeError(fn, rc)
+
+
+def make_shape(s: Spec, T: int | None = None) -> moe_shape:
+    sh = moe_shape()
+    sh.T = s.T if T is None else T
+    sh.H, sh.E, sh.topk, sh.I = s.H, s.E, s.k, s.I
+    sh.act_dtype, sh.xq_dtype = _DT[s.act], _DT[s.xq]
+    sh.weight_dtype, sh.h_dtype, sh.y_dtype, sh.out_dtype = _DT[s.weight], _DT[s.h], _DT[s.y], _DT[s.out]
+    sh.renorm, sh.identity_experts = s.renorm, s.identity
+    sh.cap_rows = s.cap_rows
+    sh.quant_block, sh.flags = 128, 0
+    return sh
+
+
+# ------------------------------------------------------------ raw C calls --
+
+def moe_workspace_bytes(shape: moe_shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_workspace_bytes", lib().moe_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def moe_workspace_init(shape: moe_shape, ws: torch.Tensor, stream=None) -> None:
+    _check("moe_workspace_init", lib().moe_workspace_init(ctypes.byref(shape), _ptr(ws),
+                                                         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route(shape, logits, topk_idx, topk_w, ws, stream=None) -> None:
+    _check("moe_route", lib().moe_route(ctypes.byref(shape), _ptr(logits), _ptr(topk_idx),
+                                        _ptr(topk_w), _ptr(ws), _stream(stream)))
+
+
+def moe_dispatch(shape, x, topk_idx, ws, bufs: moe_dispatch_bufs, stream=None) -> None:
+    _check("moe_dispatch", lib().moe_dispatch(ctypes.byref(shape), _ptr(x), _ptr(topk_idx),
+                                              _ptr(ws), ctypes.byref(bufs), _stream(stream)))
+
+
+def moe_grouped_ffn(shape, bufs: moe_dispatch_bufs, w: moe_weights, ws, y, stream=None) -> None:
+    _check("moe_grouped_ffn", lib().moe_grouped_ffn(ctypes.byref(shape), ctypes.byref(bufs),
+                                                    ctypes.byref(w), _ptr(ws), _ptr(y),
+                                                    _stream(stream)))
+
+
+def moe_combine(shape, bufs: moe_dispatch_bufs, y, topk_w, ws, out, stream=None) -> None:
+    _check("moe_combine", lib().moe_combine(ctypes.byref(shape), ctypes.byref(bufs), _ptr(y),
+                                            _ptr(topk_w), _ptr(ws), _ptr(out), _stream(stream)))
+
+
+def moe_layer(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe_dispatch_bufs, y, ws,
+              out, stream=None) -> None:
+    _check("moe_layer", lib().moe_layer(ctypes.byref(shape), _ptr(x), _ptr(logits),
+                                        ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
+                                        ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
+                                        _stream(stream)))
+
+
+def moe_poll_status(ws, stream=None) -> int:
+    return int(lib().moe_poll_status(_ptr(ws), _stream(stream)))
+
+
+def moe_status_string(code: int) -> str:
+    return lib().moe_status_string(int(code)).decode()
+
+
+# ------------------------------------------------------------ convenience --
+
+@dataclass
+class Buffers:
+    """Device buffers of one layer (torch tensors; marshalling helpers only)."""
+    shape: moe_shape
+    spec: Spec
+    ws: torch.Tensor
+    topk_idx: torch.Tensor
+    topk_w: torch.Tensor
+    xq: torch.Tensor
+    xs: torch.Tensor | None
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    row_src: torch.Tensor
+    pos: torch.Tensor
+    hq: torch.Tensor | None
+    hs: torch.Tensor | None
+    y: torch.Tensor | None
+    out: torch.Tensor
+
+    def dispatch_bufs(self) -> moe_dispatch_bufs:
+        b = moe_dispatch_bufs()
+        b.xq, b.xs = self.xq.data_ptr(), (self.xs.data_ptr() if self.xs is not None else 0)
+        b.counts, b.offsets = self.counts.data_ptr(), self.offsets.data_ptr()
+        b.row_src, b.pos = self.row_src.data_ptr(), self.pos.data_ptr()
+        b.hq = self.hq.data_ptr() if self.hq is not None else 0
+        b.hs = self.hs.data_ptr() if self.hs is not None else 0
+        return b
+
+
+def alloc_buffers(s: Spec, device="cuda", T: int | None = None, stream=None) -> Buffers:
+    """Allocate every buffer the layer writes (through torch) and initialise
+    the workspace."""
+    sh = make_shape(s, T)
+    T = sh.T
+    cap = s.cap_rows if s.cap_rows else max(128, -(-T // 128) * 128)
+    rows = s.E * cap
+    nws = moe_workspace_bytes(sh)
+    ws = torch.empty(nws, dtype=torch.uint8, device=device)
+    z = dict(device=device)
+    bufs = Buffers(
+        shape=sh, spec=s, ws=ws,
+        topk_idx=torch.empty((T, s.k), dtype=torch.int32, **z),
+        topk_w=torch.empty((T, s.k), dtype=torch.float32, **z),
+        xq=torch.empty((rows, s.H), dtype=_TORCH[s.xq], **z),
+        xs=torch.empty((rows, s.H // 128), dtype=torch.float32, **z) if s.xq == E4M3 else None,
+        counts=torch.empty(s.E, dtype=torch.int32, **z),
+        offsets=torch.empty(s.E, dtype=torch.int32, **z),
+        row_src=torch.full((rows,), -1, dtype=torch.int32, **z),
+        pos=torch.empty(T * s.k, dtype=torch.int32, **z),
+        hq=None if s.identity else torch.empty((rows, s.I), dtype=_TORCH[s.h], **z),
+        hs=torch.empty((rows, s.I // 128), dtype=torch.float32, **z)
+        if (not s.identity and s.h == E4M3) else None,
+        y=None if s.identity else torch.empty((rows, s.H), dtype=_TORCH[s.y], **z),
+        out=torch.empty((T, s.H), dtype=_TORCH[s.out], **z),
+    )
+    moe_workspace_init(sh, ws, stream)
+    return bufs
+
+
+def weights_struct(inp: dict) -> moe_weights:
+    w = moe_weights()
+    w.w_gate, w.w_up, w.w_down = (inp["w_gate"].data_ptr(), inp["w_up"].data_ptr(),
+                                  inp["w_down"].data_ptr())
+    for k in ("s_gate", "s_up", "s_down"):
+        t = inp.get(k)
+        setattr(w, k, t.data_ptr() if t is not None else 0)
+    return w
+
+
+def run_layer(b: Buffers, inp: dict, stream=None) -> None:
+    """Enqueue one whole layer (moe_layer) on the current stream."""
+    w = weights_struct(inp) if not b.spec.identity else moe_weights()
+    moe_layer(b.shape, inp["x"], inp["logits"], w, b.topk_idx, b.topk_w, b.dispatch_bufs(), b.y,
+              b.ws, b.out, stream)
+
+
+# kernels the library launches per stage (mirrors the launch plan in csrc/)
+_FFN_KERNELS = {F32: 2, BF16: 2, E4M3: 2}
+
+
+def kernels_per_layer(s: Spec) -> int:
+    """route + dispatch + grouped FFN + combine launches of one moe_layer."""
+    return 3 + (0 if s.identity else _FFN_KERNELS[s.weight])

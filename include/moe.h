@@ -1,0 +1,252 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) Mixture-of-Experts layer library.
+ *
+ * One MoE layer on one GPU, as four stages:
+ *
+ *   moe_route        router logits -> top-k experts and weights per token
+ *   moe_dispatch     one pass: each (token, slot) pair claims a row of its
+ *                    expert's window by atomic counter, quantises/copies the
+ *                    token there and publishes per-tile sentinels
+ *   moe_grouped_ffn  every expert's SwiGLU FFN over its rows, read in place
+ *   moe_combine      top-k weighted gather-reduce back to token order
+ *
+ * and moe_layer, which enqueues all four. The stage split follows the pages:
+ * an MoE layer is token dispatch, grouped GEMMs and a combine (GC-MoE feed
+ * item, "Key points"; GC-MoE explainer, "Why Expert Parallelism Is
+ * Inefficient in MoE Decoding"); dispatch pushes tokens into per-expert
+ * windows without first exchanging counts, and the grouped GEMMs read them in
+ * place rather than from a per-expert copy (NVLinkOneSided abstract); only
+ * counts, offsets and synchronisation metadata are kept as control state
+ * (Ascend relay-buffer-free report, abstract).
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" must be device memory of the current CUDA
+ *    device; pointers marked "host" must be host memory. The caller owns all
+ *    memory. The library allocates nothing and keeps no per-call global state:
+ *    everything a call needs between kernels lives in the caller's workspace.
+ *  - All work is enqueued asynchronously on `stream` (0 = legacy default
+ *    stream). Calls on different workspaces may run concurrently.
+ *  - Argument checks run on the host before anything is enqueued; on failure
+ *    the call returns MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED and enqueues
+ *    nothing. A failing CUDA launch returns MOE_ERR_CUDA.
+ *  - Errors found on the device (capacity overflow, non-finite logits, a wait
+ *    that ran out of time) are latched into the workspace, first error wins,
+ *    and read back by moe_poll_status. The library never traps, aborts or
+ *    prints.
+ *  - All device buffers must be 16-byte aligned; rows are dense (no padding).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_dtype {
+  MOE_F32 = 0,   /* IEEE binary32 */
+  MOE_BF16 = 1,  /* bfloat16 */
+  MOE_E4M3 = 2   /* OCP FP8 E4M3 with power-of-two fp32 block scales */
+} moe_dtype;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or workspace */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented dtype combination */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_CAPACITY = 4,     /* an expert received more pairs than cap_rows */
+  MOE_ERR_TIMEOUT = 5,      /* a bounded device wait gave up */
+  MOE_ERR_NONFINITE = 6     /* router logits held NaN or Inf */
+} moe_status;
+
+/*
+ * Problem description.
+ *
+ * T tokens of hidden size H, E experts of intermediate size I, top-k routing.
+ * Supported dtype combinations (act, xq, weight, h, y, out):
+ *   fp32 layer      F32,  F32,  F32,  F32,  F32,  F32
+ *   bf16 layer      BF16, BF16, BF16, BF16, BF16, BF16
+ *   fp8 layer       BF16, E4M3, E4M3, E4M3, BF16, BF16
+ *   identity experts (identity_experts = 1): act BF16/F32, xq any, out BF16/F32;
+ *                   weight/h/y ignored, moe_grouped_ffn is a no-op.
+ * H must be a multiple of 16 (of quant_block = 128 when xq is E4M3); with
+ * experts (identity_experts = 0) H and I must be multiples of 128. E <= 1024.
+ * cap_rows, when given, must be a multiple of 128.
+ * Routing weights are the softmax over all E logits of the selected experts,
+ * renormalised over the k selected ones when renorm = 1.
+ */
+typedef struct moe_shape {
+  int64_t T;              /* tokens, >= 0 */
+  int64_t H;              /* hidden size */
+  int64_t E;              /* experts, 1..65535 */
+  int64_t topk;           /* experts per token, 1..min(E, 32) */
+  int64_t I;              /* expert intermediate size */
+  int32_t act_dtype;      /* dtype of x */
+  int32_t xq_dtype;       /* dtype tokens are stored in inside expert windows */
+  int32_t weight_dtype;   /* dtype of W_gate/W_up/W_down */
+  int32_t h_dtype;        /* dtype of the SwiGLU output h */
+  int32_t y_dtype;        /* dtype of expert outputs y */
+  int32_t out_dtype;      /* dtype of the layer output */
+  int32_t renorm;         /* 1: renormalise the k weights to sum to 1 */
+  int32_t identity_experts; /* 1: every expert returns its input (no FFN) */
+  int64_t cap_rows;       /* rows per expert window; 0 = round_up(T, 128) */
+  int32_t quant_block;    /* must be 128 */
+  int32_t flags;          /* reserved, must be 0 */
+} moe_shape;
+
+/*
+ * Expert-major buffers written by moe_dispatch and moe_grouped_ffn (all device,
+ * caller-owned). cap = cap_rows (or its default); rows = E * cap. Expert e owns
+ * rows [e * cap, e * cap + counts[e]).
+ *   xq      [rows, H]        tokens in xq_dtype
+ *   xs      [rows, H/128]    fp32 power-of-two scales (E4M3 xq only, else NULL)
+ *   counts  [E]   int32      rows filled per expert (bit-exact routing counts)
+ *   offsets [E]   int32      first row of each expert window (= e * cap)
+ *   row_src [rows] int32     row -> pair id t*topk + j (rows past counts[e]
+ *                            are left as they were)
+ *   pos     [T*topk] int32   pair id -> row, or -1 if it was not placed
+ *   hq      [rows, I]        SwiGLU output in h_dtype (NULL for identity experts)
+ *   hs      [rows, I/128]    fp32 scales (E4M3 h only, else NULL)
+ * The order of rows inside an expert window is not deterministic; the set of
+ * pairs per expert is.
+ */
+typedef struct moe_dispatch_bufs {
+  void* xq;
+  float* xs;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* row_src;
+  int32_t* pos;
+  void* hq;
+  float* hs;
+} moe_dispatch_bufs;
+
+/*
+ * Expert weights (device, read only), row-major and K-major:
+ *   w_gate, w_up [E, I, H]; w_down [E, H, I], in weight_dtype.
+ *   E4M3 weights carry one fp32 scale per 128 x 128 block:
+ *   s_gate, s_up [E, I/128, H/128]; s_down [E, H/128, I/128]. Scales must be
+ *   powers of two (the tensor cores apply them as 8-bit exponents). NULL for
+ *   other weight dtypes.
+ */
+typedef struct moe_weights {
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+} moe_weights;
+
+/* Workspace size in bytes for `shape` (host only, enqueues nothing). */
+MOE_API moe_status moe_workspace_bytes(const moe_shape* shape, size_t* bytes);
+
+/*
+ * Prepare a workspace of at least moe_workspace_bytes bytes (device): zeroes
+ * the counters, the sentinels and the error word, and starts the epoch at 1.
+ * Must be called once before the first use of a workspace, and again before
+ * reusing it for a different shape.
+ */
+MOE_API moe_status moe_workspace_init(const moe_shape* shape, void* ws, size_t bytes,
+                              moe_stream_t stream);
+
+/*
+ * Routing (softmax then top-k). Reading of the pages: tokens are sent to
+ * experts according to the gating result (GC-MoE explainer, "Why Expert
+ * Parallelism Is Inefficient in MoE Decoding"); the rule itself is softmax
+ * over the E router logits, top-k on the logits (the lower expert index wins
+ * a tie), slots ordered by descending logit.
+ *   logits   [T, E] fp32, device
+ *   topk_idx [T, topk] int32, device (out)
+ *   topk_w   [T, topk] fp32, device (out)
+ *   ws       workspace (error word)
+ * A non-finite logit latches MOE_ERR_NONFINITE; that token's outputs are
+ * unspecified.
+ */
+MOE_API moe_status moe_route(const moe_shape* shape, const float* logits, int32_t* topk_idx,
+                     float* topk_w, void* ws, moe_stream_t stream);
+
+/*
+ * One-pass dispatch (NVLinkOneSided abstract: tokens are pushed into the
+ * destination windows with no metadata exchanged first; GC-MoE explainer,
+ * "Three-Node CUDA Graph and token-ring Handshake": the producer publishes
+ * filled ring blocks the consumer polls).
+ *   x        [T, H] act_dtype, device
+ *   topk_idx [T, topk] int32, device (experts must be in [0, E) and distinct
+ *            per token)
+ *   bufs     xq, xs, counts, offsets, row_src, pos are written
+ * Each pair claims row e*cap + atomicAdd(count[e], 1); E4M3 rows are
+ * quantised per 128 values with the smallest power-of-two scale that keeps
+ * the block within +-448. A pair that finds its expert full is not placed,
+ * pos = -1, and MOE_ERR_CAPACITY is latched. Every completed 128-row tile
+ * (and, when the last token is done, every partial tile) gets a sentinel.
+ */
+MOE_API moe_status moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                        void* ws, const moe_dispatch_bufs* bufs, moe_stream_t stream);
+
+/*
+ * Grouped expert FFN over the dispatched rows, read in place (NVLinkOneSided
+ * abstract; GC-MoE feed item, "Full text": block-scaled tcgen05 MMA with fused
+ * SwiGLU and requantisation). For every expert e and every filled row r:
+ *   h = silu(xq_r W_gate[e]^T) * (xq_r W_up[e]^T), stored as h_dtype in bufs->hq
+ *       (E4M3: requantised per 128 values like dispatch, scales in bufs->hs)
+ *   y_r = h W_down[e]^T, stored as y_dtype.
+ *   bufs  dispatch outputs (read) and hq/hs (written)
+ *   w     expert weights
+ *   y     [E*cap, H] y_dtype, device (out; rows past counts[e] untouched)
+ * Work starts per tile as its sentinel is found set; waits are bounded and
+ * latch MOE_ERR_TIMEOUT.
+ */
+MOE_API moe_status moe_grouped_ffn(const moe_shape* shape, const moe_dispatch_bufs* bufs,
+                           const moe_weights* w, void* ws, void* y, moe_stream_t stream);
+
+/*
+ * Weighted combine (Ascend report abstract: outputs are read straight from
+ * the expert windows, no output-restoration buffer):
+ *   out[t] = sum_{j < topk} topk_w[t, j] * y[pos[t*topk + j]]
+ * summed in slot order in fp32 and rounded once to out_dtype. With identity
+ * experts the rows are the dispatched tokens themselves (xq, dequantised with
+ * xs) and y may be NULL. Pairs with pos = -1 contribute nothing.
+ *   bufs   pos (and xq/xs for identity experts)
+ *   y      [E*cap, H] y_dtype, device
+ *   topk_w [T, topk] fp32, device
+ *   out    [T, H] out_dtype, device
+ */
+MOE_API moe_status moe_combine(const moe_shape* shape, const moe_dispatch_bufs* bufs, const void* y,
+                       const float* topk_w, void* ws, void* out, moe_stream_t stream);
+
+/*
+ * The whole layer: moe_route, moe_dispatch, moe_grouped_ffn, moe_combine
+ * enqueued in that order on `stream`. Intermediates go to the caller's
+ * buffers (topk_idx/topk_w [T, topk], bufs, y) so that they can be inspected.
+ */
+MOE_API moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits,
+                     const moe_weights* w, int32_t* topk_idx, float* topk_w,
+                     const moe_dispatch_bufs* bufs, void* y, void* ws, void* out,
+                     moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, returns the first device error latched in `ws`
+ * since the last poll (MOE_OK if none) and clears it.
+ */
+MOE_API moe_status moe_poll_status(void* ws, moe_stream_t stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,76 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/moe.h declares, sizes workspaces and rejects bad
+arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from combine_softmax_top_b200 import moe
+from combine_softmax_top_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_python_exports():
+    assert _declared() == sorted(moe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = moe.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in range(7):
+        assert moe.moe_status_string(code)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skew", "sweep"])
+def test_workspace_bytes(name):
+    s = W.spec(name)
+    n = moe.moe_workspace_bytes(moe.make_shape(s))
+    assert n > 256 and n % 256 == 0
+
+
+def test_workspace_grows_with_capacity():
+    s = W.spec("decode")
+    a = moe.moe_workspace_bytes(moe.make_shape(s))
+    b = moe.moe_workspace_bytes(moe.make_shape(s.with_(cap_rows=1024)))
+    assert b > a
+
+
+@pytest.mark.parametrize("field,value", [
+    ("topk", 0), ("topk", 33), ("E", 0), ("H", 100), ("quant_block", 64), ("flags", 1),
+    ("cap_rows", 100), ("renorm", 2), ("T", -1), ("act_dtype", 7),
+])
+def test_invalid_shapes_rejected_on_host(field, value):
+    sh = moe.make_shape(W.spec("decode"))
+    setattr(sh, field, value)
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 1
+    # every entry point checks the shape first, before any CUDA call
+    assert moe.lib().moe_route(ctypes.byref(sh), None, None, None, None, None) == 1
+
+
+def test_unsupported_dtype_combination():
+    sh = moe.make_shape(W.spec("decode"))
+    sh.h_dtype = moe.MOE_BF16   # fp8 weights with a bf16 h is not a supported layer
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 2
+
+
+def test_null_shape_and_output():
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(None, ctypes.byref(n)) == 1
+    sh = moe.make_shape(W.spec("tiny"))
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), None) == 1
+    assert moe.lib().moe_poll_status(None, None) == 1
