@@ -5,11 +5,14 @@
 #include "moe_internal.cuh"
 
 namespace moe {
-namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+namespace {
+
 bool is_dtype(int32_t d) { return d == MOE_F32 || d == MOE_BF16 || d == MOE_E4M3; }
+
+}  // namespace
 
 // Shape and dtype checks shared by every entry point.
 moe_status check_shape(const moe_shape* s) {
@@ -48,6 +51,8 @@ moe_status check_shape(const moe_shape* s) {
   return MOE_OK;
 }
 
+namespace {
+
 moe_status make_ctx(const moe_shape* s, void* ws, moe_stream_t stream, Ctx* c) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
@@ -65,6 +70,8 @@ moe_status make_ctx(const moe_shape* s, void* ws, moe_stream_t stream, Ctx* c) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+}  // namespace
+
 moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_h) {
   if (!b) return MOE_ERR_INVALID_ARG;
   if (!b->xq || !b->counts || !b->offsets || !b->row_src || !b->pos) return MOE_ERR_INVALID_ARG;
@@ -76,6 +83,8 @@ moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_
   }
   return MOE_OK;
 }
+
+namespace {
 
 moe_status check_weights(const moe_shape* s, const moe_weights* w) {
   if (!w || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;

@@ -174,6 +174,12 @@ __device__ __forceinline__ int sf_atom_offset(int m, int b) {
   return (m & 31) * 16 + (m >> 5) * 4 + b;
 }
 
+// ---- host-side argument checks (moe_api.cu) ---------------------------------
+
+bool aligned16(const void* p);
+moe_status check_shape(const moe_shape* s);
+moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_h);
+
 // ---- launchers (host, internal) --------------------------------------------
 
 struct Ctx {

@@ -25,7 +25,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CAPACITY", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_NONFINITE"}
 
 EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
-           "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_poll_status", "moe_status_string")
+           "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_poll_status", "moe_status_string",
+           "moe_dispatch_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "moe_layer": [S, P, P, ctypes.POINTER(moe_weights), P, P,
                           ctypes.POINTER(moe_dispatch_bufs), P, P, P, P],
             "moe_poll_status": [P, P],
+            "moe_dispatch_noalloc": [S, P, P, ctypes.POINTER(moe_dispatch_bufs), P],
             "moe_status_string": [ctypes.c_int],
         }
         for name, args in sig.items():
@@ -160,6 +162,14 @@ def moe_layer(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe_disp
                                         ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
                                         ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
                                         _stream(stream)))
+
+
+def moe_dispatch_noalloc(shape, x, topk_idx, bufs: moe_dispatch_bufs, stream=None) -> None:
+    """moe_dispatch for callers that cannot supply a workspace (the library's
+    fixed device array is used instead; see include/moe.h)."""
+    _check("moe_dispatch_noalloc", lib().moe_dispatch_noalloc(ctypes.byref(shape), _ptr(x),
+                                                              _ptr(topk_idx), ctypes.byref(bufs),
+                                                              _stream(stream)))
 
 
 def moe_poll_status(ws, stream=None) -> int:

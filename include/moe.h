@@ -237,6 +237,27 @@ MOE_API moe_status moe_layer(const moe_shape* shape, const void* x, const float*
                      moe_stream_t stream);
 
 /*
+ * moe_dispatch without a workspace argument, for callers that may not
+ * allocate device memory where they dispatch (an engine that hands all device
+ * memory to its own pool at start-up and forbids cudaMalloc while serving, or
+ * a latency-bound decode loop that cannot afford the device synchronisation
+ * an allocation brings). The pages have no counterpart of this call.
+ *
+ * Arguments and outputs are those of moe_dispatch (bufs: xq, xs, counts,
+ * offsets, row_src, pos). The dispatch kernel's own state lives instead in a
+ * fixed 4 MiB array of device memory inside the library, which every GPU that
+ * loads the library holds until the process exits; a shape whose workspace
+ * (moe_workspace_bytes) exceeds 4 MiB is rejected with MOE_ERR_INVALID_ARG.
+ * The first call on each device looks up that array's device address (with
+ * the device current), so make it before any stream capture. Every call
+ * clears what the kernel needs zeroed, then dispatches; calls that overlap on
+ * the GPU share the array and race. Device-detected errors are not reported
+ * through a workspace: a pair that could not be placed has pos = -1.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                                        const moe_dispatch_bufs* bufs, moe_stream_t stream);
+
+/*
  * Synchronises `stream`, returns the first device error latched in `ws`
  * since the last poll (MOE_OK if none) and clears it.
  */
