@@ -38,6 +38,7 @@ struct Args {
   int act, xq_dtype;
   moe_dispatch_bufs b;
   Ws ws;
+  uint8_t* xsf;        // scale atoms for the block-scaled MMA (NULL: not written)
   int64_t set_words;
 };
 
@@ -64,7 +65,7 @@ __device__ __forceinline__ void load16(const void* x, int act, int64_t off, floa
 __device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e, int tile,
                              int rows) {
   st_release(a.ws.sentinel + (int64_t)e * a.tpe + tile, (epoch << 8) | (uint32_t)rows);
-  const uint32_t slot = atomicAdd(set + a.E + a.E * a.tpe + kRingHead, 1u);
+  const uint32_t slot = atomicAdd(set_misc(set) + kRingHead, 1u);
   st_release64(a.ws.ring + slot,
                ((unsigned long long)epoch << 32) | ((unsigned long long)e << 16) | (unsigned)tile);
 }
@@ -81,9 +82,9 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
   const uint32_t epoch = s_epoch;
   uint32_t* set = a.ws.set[epoch & 1];
   uint32_t* next = a.ws.set[(epoch + 1) & 1];
-  uint32_t* count = set;
-  uint32_t* fill = set + a.E;
-  uint32_t* misc = set + a.E + (int64_t)a.E * a.tpe;
+  uint32_t* count = set_count(set);
+  uint32_t* fill = set_fill(set, a.E);
+  uint32_t* misc = set_misc(set);
 
   // zero this CTA's share of the next counter set
   {
@@ -154,10 +155,12 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
           *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
           if (leader) {
             a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
-            const int tile = row / kTileRows;   // global tile id e * tpe + local (cap % 128 == 0)
-            const int m = row % kTileRows;
-            a.ws.xsf[((int64_t)tile * ((a.H + 511) / 512) + blk / 4) * kSfAtomBytes +
-                     sf_atom_offset(m, blk & 3)] = (uint8_t)(p + 127);
+            if (a.xsf) {
+              const int tile = row / kTileRows;   // global tile id e * tpe + local (cap % 128 == 0)
+              const int m = row % kTileRows;
+              *reinterpret_cast<uint32_t*>(a.xsf + ((int64_t)tile * (a.H / kQBlock) + blk) * kSfAtomBytes +
+                                           sf_atom_offset(m)) = (uint32_t)(p + 127) * 0x01010101u;
+            }
           }
         }
       } else if (live) {
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
 }  // namespace
 
 cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
-                            const moe_dispatch_bufs& b) {
+                            const moe_dispatch_bufs& b, bool write_sf) {
   Args a;
   a.x = x;
   a.idx = idx;
@@ -245,6 +248,7 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
   a.xq_dtype = c.s.xq_dtype;
   a.b = b;
   a.ws = c.ws;
+  a.xsf = write_sf && c.s.xq_dtype == MOE_E4M3 ? c.ws.xsf : nullptr;
   a.set_words = (int64_t)c.L.set_words;
   const int grid = a.T > 0 ? a.T : 1;
   dispatch_kernel<<<grid, kThreads, 0, c.stream>>>(a);

@@ -71,7 +71,9 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x
   Ctx c;
   c.s = *shape;
   c.L = make_layout(*shape);
-  if (c.L.total > kNoAllocScratchBytes) return MOE_ERR_INVALID_ARG;   // too big for the fixed scratch
+  // counters, sentinels and ring only: the scale atoms for the tensor-core
+  // FFN are not written on this path
+  if (c.L.off_xsf > kNoAllocScratchBytes) return MOE_ERR_INVALID_ARG;   // too big for the fixed scratch
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   c.ws = ws_view(scratch, c.L);
@@ -84,5 +86,5 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x
   clear_scratch_kernel<<<(unsigned)std::min<size_t>((words + 255) / 256, 256), 256, 0, c.stream>>>(
       (uint32_t*)scratch, words);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  return launch_dispatch(c, x, topk_idx, *bufs) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_dispatch(c, x, topk_idx, *bufs, /*write_sf=*/false) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -26,7 +26,6 @@ struct Args {
   int xq_dt, w_dt, h_dt, y_dt;
   Ws ws;
   uint8_t* hsf;
-  int64_t igroups;
 };
 
 __device__ __forceinline__ float ld_act(const void* p, int dt, int64_t i) {
@@ -81,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
   const int NF = DOWN ? a.H : a.I;  // output features
   const int nslices = NF / kF;
   const uint32_t epoch = a.ws.hdr->epoch_cur;
-  const uint32_t* misc = a.ws.set[epoch & 1] + a.E + (int64_t)a.E * a.tpe;
+  const uint32_t* misc = set_misc(a.ws.set[epoch & 1]);
   const uint32_t total = ld_acquire(misc + kRingTotal);
   const void* xin = DOWN ? a.hq : a.xq;
   const float* xsc = DOWN ? a.hs : a.xs;
@@ -187,8 +186,9 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
             if (f == 0) {
               a.hs[row * (a.I / kQBlock) + slice] = exp2i(p);
               if (a.hsf)
-                a.hsf[((int64_t)(row / kTileRows) * a.igroups + slice / 4) * kSfAtomBytes +
-                      sf_atom_offset((int)(row % kTileRows), slice & 3)] = (uint8_t)(p + 127);
+                *reinterpret_cast<uint32_t*>(a.hsf + ((int64_t)(row / kTileRows) * (a.I / kQBlock) + slice) *
+                                                         kSfAtomBytes + sf_atom_offset((int)(row % kTileRows))) =
+                    (uint32_t)(p + 127) * 0x01010101u;
             }
           }
         }
@@ -220,7 +220,6 @@ cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_
   a.xq_dt = c.s.xq_dtype; a.w_dt = c.s.weight_dtype; a.h_dt = c.s.h_dtype; a.y_dt = c.s.y_dtype;
   a.ws = c.ws;
   a.hsf = c.s.h_dtype == MOE_E4M3 ? c.ws.hsf : nullptr;
-  a.igroups = c.L.igroups;
   const int grid = c.num_sms * 4;
   ffn_simt_kernel<false><<<grid, kThreads, 0, c.stream>>>(a);
   cudaError_t err = cudaGetLastError();

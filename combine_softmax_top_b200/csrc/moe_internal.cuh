@@ -23,13 +23,17 @@ constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
 // [header 256 B][counter set 0][counter set 1][sentinels][ring][xsf][hsf]
 //
 // header : epoch_next, epoch_cur, error, error_info (u32 each)
-// set    : count[E] | fill[E*tpe] | misc[8] (ring_head, done, ring_total, ...)
+// set    : misc[8] (ring_head, done, ring_total, ...) | count[E] |
+//          fill[E*tpe] | hdone[E*tpe]
 //          two sets are used alternately by consecutive dispatches; each
 //          dispatch zeroes the set the following dispatch will use.
+//          hdone[slot] counts the finished gate/up slices of ring slot `slot`.
 // sentinel[E*tpe] u32 : (epoch << 8) | rows of a published tile
 // ring[E*tpe] u64     : (epoch << 32) | (e << 16) | tile, in publication order
 // xsf / hsf           : UE8M0 scale atoms of xq / hq for the block-scaled MMA,
-//                       [tile][group of 4 blocks][512 B]
+//                       [tile][128-value block][512 B]; row m of the tile owns
+//                       the 32-bit word at (m % 32) * 16 + (m / 32) * 4, all
+//                       four bytes holding the block's exponent
 struct Header {
   uint32_t epoch_next;
   uint32_t epoch_cur;
@@ -43,7 +47,7 @@ enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kMiscWords = 8 };
 
 struct Layout {
   int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles = E * tpe
-  int64_t hgroups, igroups;                 // ceil(H/512), ceil(I/512)
+  int64_t hblocks, iblocks;                 // H/128, I/128 (scale atoms per tile)
   size_t set_words;                         // u32 words of one counter set
   size_t off_set[2], off_sentinel, off_ring, off_xsf, off_hsf, total;
 };
@@ -63,9 +67,9 @@ inline Layout make_layout(const moe_shape& s) {
   L.cap = default_cap(s);
   L.tpe = ceil_div(L.cap, kTileRows);
   L.tiles = L.E * L.tpe;
-  L.hgroups = ceil_div(L.H, 4 * kQBlock);
-  L.igroups = ceil_div(L.I, 4 * kQBlock);
-  L.set_words = (size_t)(L.E + L.tiles + kMiscWords);
+  L.hblocks = ceil_div(L.H, kQBlock);
+  L.iblocks = ceil_div(L.I, kQBlock);
+  L.set_words = (size_t)(kMiscWords + L.E + 2 * L.tiles);
   size_t off = sizeof(Header);
   for (int i = 0; i < 2; ++i) {
     L.off_set[i] = off;
@@ -76,10 +80,10 @@ inline Layout make_layout(const moe_shape& s) {
   L.off_ring = off;
   off = align_up(off + (size_t)L.tiles * 8, 256);
   L.off_xsf = off;
-  if (s.xq_dtype == MOE_E4M3) off = align_up(off + (size_t)L.tiles * L.hgroups * kSfAtomBytes, 256);
+  if (s.xq_dtype == MOE_E4M3) off = align_up(off + (size_t)L.tiles * L.hblocks * kSfAtomBytes, 256);
   L.off_hsf = off;
   if (s.h_dtype == MOE_E4M3 && !s.identity_experts)
-    off = align_up(off + (size_t)L.tiles * L.igroups * kSfAtomBytes, 256);
+    off = align_up(off + (size_t)L.tiles * L.iblocks * kSfAtomBytes, 256);
   L.total = off;
   return L;
 }
@@ -168,10 +172,18 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
   return __half2float(__half(hr));
 }
 
-// Byte offset of (row m of a 128-row tile, block b of a 4-block group) inside
-// one scale-factor atom: 32 lanes x 16 bytes, lane m % 32, word m / 32, byte b.
-__device__ __forceinline__ int sf_atom_offset(int m, int b) {
-  return (m & 31) * 16 + (m >> 5) * 4 + b;
+// Byte offset of row m's 32-bit word inside one scale-factor atom of a
+// 128-row tile: 32 lanes x 16 bytes, lane m % 32, word m / 32.
+__device__ __forceinline__ int sf_atom_offset(int m) {
+  return (m & 31) * 16 + (m >> 5) * 4;
+}
+
+// Counter-set views.
+__device__ __forceinline__ uint32_t* set_misc(uint32_t* set) { return set; }
+__device__ __forceinline__ uint32_t* set_count(uint32_t* set) { return set + kMiscWords; }
+__device__ __forceinline__ uint32_t* set_fill(uint32_t* set, int E) { return set + kMiscWords + E; }
+__device__ __forceinline__ uint32_t* set_hdone(uint32_t* set, int E, int64_t tiles) {
+  return set + kMiscWords + E + tiles;
 }
 
 // ---- host-side argument checks (moe_api.cu) ---------------------------------
@@ -191,8 +203,9 @@ struct Ctx {
 };
 
 cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float* w);
+// write_sf: also write the e4m3 scale atoms the tensor-core FFN reads
 cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
-                            const moe_dispatch_bufs& b);
+                            const moe_dispatch_bufs& b, bool write_sf = true);
 cudaError_t launch_combine(const Ctx& c, const moe_dispatch_bufs& b, const void* y,
                            const float* topk_w, void* out);
 cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,

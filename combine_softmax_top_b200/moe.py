@@ -259,7 +259,7 @@ def run_layer(b: Buffers, inp: dict, stream=None) -> None:
 
 
 # kernels the library launches per stage (mirrors the launch plan in csrc/)
-_FFN_KERNELS = {F32: 2, BF16: 2, E4M3: 2}
+_FFN_KERNELS = {F32: 2, BF16: 1, E4M3: 1}
 
 
 def kernels_per_layer(s: Spec) -> int:
