@@ -36,6 +36,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--config", default="decode")
     p.add_argument("--T", type=int, default=None, help="override the token count")
+    p.add_argument("--E", type=int, default=None, help="override the expert count (small profiling cases)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -43,6 +44,15 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall-clock budget of the CPU oracle sample")
     return p.parse_args()
+
+
+def overrides(args) -> dict:
+    o = {}
+    if args.T:
+        o["T"] = args.T
+    if args.E:
+        o["E"] = args.E
+    return o
 
 
 def dist_env():
@@ -170,17 +180,19 @@ def ffn_flops(spec, rows):
 
 
 def recorded_traffic(kernel_tag: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel (else None)."""
-    path = os.path.join(PROFILES, "traffic.json")
+    """DRAM bytes per launch from the committed ncu summary table
+    (profiles/traffic.md), if it was taken on the current source of the
+    kernel (else None)."""
+    path = os.path.join(PROFILES, "traffic.md")
     if not os.path.exists(path):
         return None
-    rec = json.load(open(path)).get(kernel_tag)
-    if not rec:
-        return None
-    if rec.get("source_sha") != kernel_source_sha():
-        return None
-    return rec.get("dram_bytes_per_launch")
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 3 and cells[0] == kernel_tag:
+            if cells[1] != kernel_source_sha():
+                return None
+            return int(cells[2])
+    return None
 
 
 def kernel_source_sha() -> str:
@@ -208,7 +220,7 @@ def run_reference(args):
         return
     from combine_softmax_top_b200 import workloads as W
     import torch
-    spec = W.spec(args.config, **({"T": args.T} if args.T else {}))
+    spec = W.spec(args.config, **overrides(args))
     inp = W.make_inputs(spec, seed=args.seed, device="cpu")
     per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -249,7 +261,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
-    spec = W.spec(args.config, **({"T": args.T} if args.T else {}))
+    spec = W.spec(args.config, **overrides(args))
     inp = W.make_inputs(spec, seed=args.seed + rank, device=dev)
     b = moe.alloc_buffers(spec, device=dev)
     w = moe.weights_struct(inp) if not spec.identity else moe.moe_weights()

@@ -50,10 +50,21 @@ __device__ bool fetch_tile(const Args& a, uint32_t epoch, uint32_t slot, int* e,
   }
   *e = (int)((ent >> 16) & 0xFFFF);
   *tile = (int)(ent & 0xFFFF);
+  if (*e >= a.E || *tile >= a.tpe) {          // never published: a corrupt workspace
+    latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, slot);
+    return false;
+  }
   const uint32_t* sp = a.ws.sentinel + (int64_t)(*e) * a.tpe + *tile;
   while (true) {
     const uint32_t s = ld_acquire(sp);
-    if ((s >> 8) == (epoch & 0xFFFFFFu)) { *rows = (int)(s & 0xFF); return true; }
+    if ((s >> 8) == (epoch & 0xFFFFFFu)) {
+      *rows = (int)(s & 0xFF);
+      if (*rows < 1 || *rows > kTileRows) {
+        latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, slot);
+        return false;
+      }
+      return true;
+    }
     if (globaltimer() - t0 > kWaitBudgetNs) {
       latch_error(a.ws.hdr, MOE_ERR_TIMEOUT, slot);
       return false;

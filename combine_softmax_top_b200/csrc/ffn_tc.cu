@@ -119,11 +119,21 @@ __device__ bool fetch_tile(const TcParams& p, uint32_t epoch, uint32_t slot, vol
   }
   *e = (int)((ent >> 16) & 0xFFFF);
   *tile = (int)(ent & 0xFFFF);
+  if (*e >= p.E || *tile >= p.tpe) {          // never published: a corrupt workspace
+    latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x11000000u | slot);
+    *abort_flag = 1;
+    return false;
+  }
   const uint32_t* sp = p.ws.sentinel + (int64_t)(*e) * p.tpe + *tile;
   while (true) {
     const uint32_t s = ld_acquire(sp);
     if ((s >> 8) == (epoch & 0xFFFFFFu)) {
       *rows = (int)(s & 0xFF);
+      if (*rows < 1 || *rows > kTileRows) {   // never published: a corrupt workspace
+        latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x21000000u | slot);
+        *abort_flag = 1;
+        return false;
+      }
       return true;
     }
     if (*abort_flag) return false;

@@ -239,3 +239,35 @@ def test_identity_experts_return_input(T, cuda_device):
     r = oracle.moe_layer(p, raw(inp["x"]), raw(inp["logits"]))
     ref = as_f64(r["out"], "bf16")
     assert np.all(np.abs(out - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-30)
+
+
+# ------------------------------------------------------- bounded waits --
+
+def test_ffn_wait_runs_out_and_context_survives(cuda_device):
+    """Announce one more tile than dispatch published: the FFN's wait for it
+    must give up (MOE_ERR_TIMEOUT) instead of hanging, and the device must
+    stay usable."""
+    s = W.spec("decode", T=32, H=512, E=16, k=4, I=256)
+    inp = W.make_inputs(s, seed=5, device="cuda")
+    b = moe.alloc_buffers(s)
+    moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws)
+    moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, b.dispatch_bufs())
+    assert G.poll(b) == 0
+    # workspace layout: 256-byte header (epoch_next, epoch_cur, ...), then the
+    # counter sets; after the first dispatch epoch_cur = 1 -> set 1, whose
+    # third word is the published tile total
+    hdr = b.ws[:16].view(torch.int32)
+    assert int(hdr[1]) == 1
+    set_words = 8 + s.E + 2 * s.E * (s.cap // 128)
+    set1 = 256 + ((set_words * 4 + 255) // 256) * 256
+    total = b.ws[set1 + 8:set1 + 12].view(torch.int32)
+    total += 1                                   # a tile nothing will ever publish
+    torch.cuda.synchronize()
+    moe.moe_grouped_ffn(b.shape, b.dispatch_bufs(), moe.weights_struct(inp), b.ws, b.y)
+    assert G.poll(b) == 5                        # MOE_ERR_TIMEOUT
+    # the context is intact: a fresh layer runs and matches the oracle
+    b2 = G.run_stages(s, inp, layer=True)
+    assert G.poll(b2) == 0
+    p = G.oracle_problem(s, inp)
+    r = oracle.moe_layer(p, raw(inp["x"]), raw(inp["logits"]))
+    assert max_abs_rel(as_f64(raw(b2.out), "bf16"), as_f64(r["out"], "bf16")) < 2e-2
