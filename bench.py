@@ -43,6 +43,10 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall-clock budget of the CPU oracle sample")
+    p.add_argument("--report", action="store_true",
+                   help="instead of the single bench line: one JSON line per workload "
+                        "(tiny, decode, prefill, skew, dispatch+combine sweep) with per-stage "
+                        "times and roofline fractions")
     return p.parse_args()
 
 
@@ -246,6 +250,121 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+EL = {"f32": 4, "bf16": 2, "e4m3": 1}
+
+
+def route_bytes(spec):
+    return spec.T * (4 * spec.E + 8 * spec.k)
+
+
+def dispatch_bytes(spec):
+    """x read once, k rows (+ scales and scale atoms) written, pos/row_src."""
+    per_pair = spec.H * EL[spec.xq] + 8
+    if spec.xq == "e4m3":
+        per_pair += 2 * (spec.H // 128) * 4
+    return spec.T * (spec.H * EL[spec.act] + 4 * spec.k + spec.k * per_pair)
+
+
+def combine_bytes(spec):
+    """k rows gathered (identity: e4m3 rows + scales), pos and weights, out written."""
+    if spec.identity:
+        row = spec.H * EL[spec.xq] + ((spec.H // 128) * 4 if spec.xq == "e4m3" else 0)
+    else:
+        row = spec.H * EL[spec.y]
+    return spec.T * (spec.k * (row + 8) + spec.H * EL[spec.out])
+
+
+def time_layer(spec, inp, b, steps, warmup, stream, flush):
+    """Per-stage device times (ms, one row per step) through the per-stage
+    C-ABI calls, with L2 flushed before every step."""
+    import numpy as np
+    import torch
+    from combine_softmax_top_b200 import moe
+
+    w = moe.weights_struct(inp) if not spec.identity else moe.moe_weights()
+    bufs = b.dispatch_bufs()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws, stream)
+        if ev:
+            ev[1].record(stream)
+        moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, bufs, stream)
+        if ev:
+            ev[2].record(stream)
+        if not spec.identity:
+            moe.moe_grouped_ffn(b.shape, bufs, w, b.ws, b.y, stream)
+        if ev:
+            ev[3].record(stream)
+        moe.moe_combine(b.shape, bufs, b.y, b.topk_w, b.ws, b.out, stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    rc = moe.moe_poll_status(b.ws, stream)
+    if rc != 0:
+        raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
+    return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)])
+
+
+def run_report(args):
+    import numpy as np
+    import torch
+    from combine_softmax_top_b200 import moe
+    from combine_softmax_top_b200 import workloads as W
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peaks, kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    cases = [W.spec("tiny"), W.spec("decode"), W.spec("prefill"), W.spec("skew")] + \
+        [W.spec("sweep", T=t) for t in W.SWEEP_T]
+    for spec in cases:
+        inp = W.make_inputs(spec, seed=args.seed, device=dev)
+        b = moe.alloc_buffers(spec, device=dev)
+        st = time_layer(spec, inp, b, args.steps, args.warmup, stream, flush).mean(0)
+        counts = b.counts.cpu().numpy()
+        layer_ms = float(st.sum())
+        line = {"report": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k,
+                "I": None if spec.identity else spec.I, "dtype": spec.weight if not spec.identity else spec.xq,
+                "layer_us": layer_ms * 1e3, "tokens_per_s": spec.T / (layer_ms / 1e3),
+                "stage_us": {k: float(v * 1e3) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], st)},
+                "peak_source": kind}
+        rb, db, cb = route_bytes(spec), dispatch_bytes(spec), combine_bytes(spec)
+        line["route_GBps"] = rb / (st[0] / 1e3) / 1e9
+        line["dispatch_GBps"] = db / (st[1] / 1e3) / 1e9
+        line["combine_GBps"] = cb / (st[3] / 1e3) / 1e9
+        line["dispatch_frac_hbm"] = line["dispatch_GBps"] / hbm
+        line["combine_frac_hbm"] = line["combine_GBps"] / hbm
+        if spec.identity:
+            line["permutation_GBps"] = (db + cb) / ((st[1] + st[3]) / 1e3) / 1e9
+            line["permutation_frac_hbm"] = line["permutation_GBps"] / hbm
+        else:
+            abytes, touched = ffn_algorithmic_bytes(spec, counts)
+            flops = ffn_flops(spec, int(counts.sum()))
+            tc_peak = peaks["bf16_tflops"] * (2.0 if spec.weight == "e4m3" else 1.0)
+            line["ffn_GBps"] = abytes / (st[2] / 1e3) / 1e9
+            line["ffn_TFLOPs"] = flops / (st[2] / 1e3) / 1e12
+            line["ffn_frac_hbm"] = line["ffn_GBps"] / hbm
+            line["ffn_frac_tensor"] = line["ffn_TFLOPs"] / tc_peak
+            line["ffn_bound"] = "hbm" if abytes / (hbm * 1e9) >= flops / (tc_peak * 1e12) else "tensor"
+            line["touched_experts"] = touched
+        print(json.dumps(line), flush=True)
+        del inp, b
+        torch.cuda.empty_cache()
+
+
 # ------------------------------------------------------------ ours --
 
 def run_ours(args):
@@ -421,6 +540,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.report:
+        run_report(args)
     else:
         run_ours(args)
 

@@ -16,7 +16,7 @@
 // All gate/up units come before all down units; a down unit waits until the
 // I/128 gate/up units of its tile have stored h (per-slot counter).
 //
-// Per CTA (192 threads): warp 0 streams K slabs of 128 bytes into a 4-stage
+// Per CTA (224 threads): warp 6 schedules jobs; warp 0 streams K slabs of 128 bytes into a 4- or 5-stage
 // shared-memory ring with TMA (weights with an evict-first hint), and for
 // e4m3 builds the weights' UE8M0 scale atoms and bulk-copies the tokens';
 // warp 1 issues tcgen05.mma (kind::f16 for bf16, kind::mxf8f6f4.block_scale
@@ -35,23 +35,36 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
-constexpr int kSlab = 128;                 // K bytes per stage (one 128-byte swizzle row)
-constexpr int kABytes = 128 * kSlab;       // 128 weight rows
-constexpr int kBBytes = 128 * kSlab;       // up to 128 token rows
-constexpr int kOffA1 = kABytes;
-constexpr int kOffB = 2 * kABytes;
-constexpr int kOffSfa0 = 2 * kABytes + kBBytes;
-constexpr int kOffSfa1 = kOffSfa0 + kSfAtomBytes;
-constexpr int kOffSfb = kOffSfa1 + kSfAtomBytes;
-constexpr int kStageStride = 51200;        // 50688 rounded up to 1024
-static_assert(kOffSfb + kSfAtomBytes <= kStageStride, "stage layout");
-constexpr int kBarOffset = kStages * kStageStride;
-constexpr int kSmemBytes = kBarOffset + 1024 /* barriers, flags, reductions */ + 1024 /* alignment slack */;
+constexpr int kThreads = 224;   // warps: 0 TMA, 1 MMA, 2-5 epilogue, 6 scheduler
+constexpr int kUQ = 8;          // unit-queue depth
+constexpr int kSlab = 128;      // K bytes per slab (one 128-byte swizzle row)
+constexpr int kABytes = 128 * kSlab;   // 128 weight rows of one slab
+constexpr int kMaxDynSmem = 232448;    // 227 KB per CTA
+constexpr int kCtlBytes = 1024;        // barriers, unit queue, flags, reductions (664 B used)
+
+// Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
+// A0 | A1 | B (kBRows x 128 B, or two slabs of N rows) | SFA0 | SFA1 | SFB0 | SFB1
+template <int kBRows>
+struct Stage {
+  static constexpr int kOffA1 = kABytes;
+  static constexpr int kOffB = 2 * kABytes;
+  static constexpr int kOffSfa0 = kOffB + kBRows * kSlab;
+  static constexpr int kOffSfa1 = kOffSfa0 + kSfAtomBytes;
+  static constexpr int kOffSfb0 = kOffSfa1 + kSfAtomBytes;
+  static constexpr int kOffSfb1 = kOffSfb0 + kSfAtomBytes;
+  static constexpr int kStride = (kOffSfb1 + kSfAtomBytes + 1023) / 1024 * 1024;
+  static constexpr int kStages = (kMaxDynSmem - kCtlBytes - 1024) / kStride;
+  static constexpr int kBarOffset = kStages * kStride;
+  static constexpr int kSmemBytes = kBarOffset + kCtlBytes + 1024 /* alignment slack */;
+  static_assert(kStages >= 3, "pipeline depth");
+};
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColG = 0, kColU = 128, kColSfa0 = 256, kColSfa1 = 260, kColSfb = 264;
+// accumulators: two 128-column slots at columns 0 and 128; scale factors after
+constexpr uint32_t kColSfa0 = 256, kColSfa1 = 260, kColSfb0 = 264, kColSfb1 = 268;
+
+enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
+enum : int { kFfnGen = 3, kFfnExit = 4 };   // counter-set misc slots used here
 
 struct TcParams {
   CUtensorMap tm_wg, tm_wu, tm_wd, tm_x, tm_h;
@@ -69,20 +82,36 @@ struct TcParams {
   int64_t tiles;
 };
 
-struct Unit {
-  bool down;
-  uint32_t slot;
-  int slice;
+// One queue entry: a chunk of <= kBRows rows of one tile, for one 128-feature
+// slice, in one phase.
+struct Job {
+  int e, tile, slice, rows, row_off, kind, nslab, slot;
 };
 
-__device__ __forceinline__ Unit unit_of(uint32_t u, uint32_t n1, int n_islices, int n_hslices) {
-  Unit r;
-  r.down = u >= n1;
-  const uint32_t v = r.down ? u - n1 : u;
-  const int ns = r.down ? n_hslices : n_islices;
-  r.slot = v / ns;
-  r.slice = (int)(v % ns);
-  return r;
+__device__ __forceinline__ int4 pack_job(const Job& j) {
+  return make_int4(j.e, j.tile | (j.slice << 16),
+                   j.rows | (j.row_off << 8) | (j.kind << 16) | (j.nslab << 20), j.slot);
+}
+
+__device__ __forceinline__ Job unpack_job(int4 v) {
+  Job j;
+  j.e = v.x;
+  j.tile = v.y & 0xFFFF;
+  j.slice = (v.y >> 16) & 0xFFFF;
+  j.rows = v.z & 0xFF;
+  j.row_off = (v.z >> 8) & 0xFF;
+  j.kind = (v.z >> 16) & 0xF;
+  j.nslab = (v.z >> 20) & 0xF;
+  j.slot = v.w;
+  return j;
+}
+
+__device__ __forceinline__ int4 shfl_int4(int4 v) {
+  v.x = __shfl_sync(0xffffffffu, v.x, 0);
+  v.y = __shfl_sync(0xffffffffu, v.y, 0);
+  v.z = __shfl_sync(0xffffffffu, v.z, 0);
+  v.w = __shfl_sync(0xffffffffu, v.w, 0);
+  return v;
 }
 
 // Bounded wait on an mbarrier phase; false on timeout (latched) or abort.
@@ -168,19 +197,26 @@ __device__ __forceinline__ uint32_t ue8m0_word(float s) {
   return ((__float_as_uint(s) >> 23) & 0xFFu) * 0x01010101u;
 }
 
-template <bool kFp8>
+template <bool kFp8, int kBRows>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_constant__ TcParams p) {
+  using S = Stage<kBRows>;
+  constexpr int kStages = S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  uint8_t* ctl = smem + S::kBarOffset;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* epi_info = reinterpret_cast<int*>(tmem_slot + 4);       // ok, e, tile, rows
-  float* red = reinterpret_cast<float*>(tmem_slot + 8);        // [4 warps][16 tokens]
+  uint64_t* acc_full = empty + kStages;       // [2] per accumulator slot
+  uint64_t* acc_empty = acc_full + 2;         // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* uq_full = drain + 1;              // [kUQ] job queue
+  uint64_t* uq_empty = uq_full + kUQ;         // [kUQ]
+  static_assert((2 * kStages + 5 + 2 * kUQ) * 8 <= 256, "barriers fit before the job queue");
+  int4* uq = reinterpret_cast<int4*>(ctl + 256);               // [kUQ] packed jobs
+  float* red = reinterpret_cast<float*>(ctl + 384);            // [4 warps][16 tokens]
+  int4* epi_job = reinterpret_cast<int4*>(ctl + 640);          // job broadcast to the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 656);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 660);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -190,9 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ptx::mbar_init(full + s, 1);
       ptx::mbar_init(empty + s, 1);
     }
-    ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(acc_full + s, 1);
+      ptx::mbar_init(acc_empty + s, 1);
+    }
     ptx::mbar_init(drain, 1);
+    for (int q = 0; q < kUQ; ++q) {
+      ptx::mbar_init(uq_full + q, 1);
+      ptx::mbar_init(uq_empty + q, 3);   // producer, MMA issuer, epilogue
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -207,13 +249,70 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
 
   const uint32_t epoch = p.ws.hdr->epoch_cur;
   uint32_t* set = p.ws.set[epoch & 1];
-  const uint32_t ntiles = ld_acquire(set_misc(set) + kRingTotal);
+  uint32_t* misc = set_misc(set);
+  const uint32_t ntiles = ld_acquire(misc + kRingTotal);
+  const uint32_t gen = ld_acquire(misc + kFfnGen);   // FFN calls already made on this dispatch
   uint32_t* hdone = set_hdone(set, p.E, p.tiles);
   const uint32_t n1 = ntiles * (uint32_t)p.n_islices;
   const uint32_t total = n1 + ntiles * (uint32_t)p.n_hslices;
   Header* hdr = p.ws.hdr;
 
-  if (warp == 0) {
+  // Take job i from the queue (one lane of a consumer role).
+  auto take_job = [&](uint32_t i, Job* out) -> bool {
+    const uint32_t q = i % kUQ, ph = (i / kUQ) & 1u;
+    if (!wait_bar(uq_full + q, ph, abort_flag, hdr, 0x80000000u | q)) return false;
+    *out = unpack_job(uq[q]);
+    ptx::mbar_arrive(uq_empty + q);
+    return true;
+  };
+
+  if (warp == 6) {
+    // ---------------------------------------------------------------- scheduler
+    // Units (ring slot x 128-feature slice; all gate/up units before all down
+    // units) are dealt round-robin to the CTAs. For each unit the scheduler
+    // resolves the tile (ring entry + sentinel), waits for a down unit's h,
+    // splits the tile into chunks of <= kBRows rows and queues them.
+    if (lane == 0) {
+      uint32_t i = 0;
+      bool good = true;
+      auto push = [&](const Job& j) -> bool {
+        const uint32_t q = i % kUQ, ph = (i / kUQ) & 1u;
+        if (!wait_bar(uq_empty + q, ph ^ 1u, abort_flag, hdr, 0x90000000u | q)) return false;
+        uq[q] = pack_job(j);
+        ptx::mbar_arrive(uq_full + q);
+        ++i;
+        return true;
+      };
+      for (uint32_t u = blockIdx.x; good && u < total; u += gridDim.x) {
+        Job j;
+        j.kind = u >= n1 ? kKindDown : kKindGateUp;
+        const uint32_t v = j.kind == kKindDown ? u - n1 : u;
+        const int ns = j.kind == kKindDown ? p.n_hslices : p.n_islices;
+        j.slot = (int)(v / ns);
+        j.slice = (int)(v % ns);
+        int rows = 0;
+        good = fetch_tile(p, epoch, (uint32_t)j.slot, abort_flag, &j.e, &j.tile, &rows);
+        if (!good) break;
+        const int nch = (rows + kBRows - 1) / kBRows;
+        if (j.kind == kKindDown)
+          good = wait_count(hdone + j.slot, (uint32_t)(p.n_islices * nch) * (gen + 1u), abort_flag, hdr,
+                            0x30000000u | (uint32_t)j.slot);
+        for (int c = 0; good && c < nch; ++c) {
+          j.row_off = c * kBRows;
+          j.rows = min(kBRows, rows - j.row_off);
+          const int N = (j.rows + 15) & ~15;
+          j.nslab = (j.kind == kKindDown && 2 * N <= kBRows && (p.nk2 & 1) == 0) ? 2 : 1;
+          good = push(j);
+        }
+      }
+      Job end;
+      end.e = end.tile = end.slice = end.rows = end.row_off = end.slot = 0;
+      end.nslab = 1;
+      end.kind = good ? kKindEnd : kKindAbort;
+      push(end);   // bounded; consumers also stop on the abort flag
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       ptx::prefetch_tmap(&p.tm_wg);
@@ -225,73 +324,80 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     const uint64_t pol = ptx::policy_evict_first();
     uint32_t stage = 0, phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per stage: a load is outstanding / its phase parity
-    bool ok = true;
-    for (uint32_t u = blockIdx.x; ok && u < total; u += gridDim.x) {
-      const Unit un = unit_of(u, n1, p.n_islices, p.n_hslices);
-      int e = 0, tile = 0, rows = 0;
-      int good = 1;
+    for (uint32_t i = 0;; ++i) {
+      int4 raw = make_int4(0, 0, kKindAbort << 16, 0);
       if (lane == 0) {
-        good = fetch_tile(p, epoch, un.slot, abort_flag, &e, &tile, &rows);
-        if (good && un.down)
-          good = wait_count(hdone + un.slot, (uint32_t)p.n_islices, abort_flag, hdr, 0x30000000u | un.slot);
+        Job jj;
+        if (take_job(i, &jj)) raw = pack_job(jj);
         ptx::fence_proxy_async_global();   // rows written by other CTAs -> TMA reads
       }
-      good = __shfl_sync(0xffffffffu, good, 0);
-      if (!good) { ok = false; break; }
-      e = __shfl_sync(0xffffffffu, e, 0);
-      tile = __shfl_sync(0xffffffffu, tile, 0);
-      rows = __shfl_sync(0xffffffffu, rows, 0);
-      const int N = (rows + 15) & ~15;
-      const int nk = un.down ? p.nk2 : p.nk1;
-      const int arow = e * (un.down ? p.H : p.I) + un.slice * 128;
-      const int row0 = e * p.cap + tile * kTileRows;
-      const int64_t tile_g = (int64_t)e * p.tpe + tile;
-      const uint32_t tx = (un.down ? 1u : 2u) * kABytes + (uint32_t)N * kSlab + (kFp8 ? kSfAtomBytes : 0u);
-      for (int kb = 0; kb < nk; ++kb) {
+      const Job j = unpack_job(shfl_int4(raw));
+      if (j.kind >= kKindEnd) break;
+      const bool down = j.kind == kKindDown;
+      const int N = (j.rows + 15) & ~15;
+      const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
+      const int arow = j.e * (down ? p.H : p.I) + j.slice * 128;
+      const int brow = j.e * p.cap + j.tile * kTileRows + j.row_off;
+      const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
+      const uint32_t tx = (down ? (uint32_t)j.nslab : 2u) * kABytes + (uint32_t)(j.nslab * N * kSlab) +
+                          (kFp8 ? (uint32_t)j.nslab * kSfAtomBytes : 0u);
+      bool ok = true;
+      for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
         if (lane == 0) w_ok = wait_bar(empty + stage, phase ^ 1u, abort_flag, hdr, 0x40000000u | stage);
         w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
         if (!w_ok) { ok = false; break; }
         __syncwarp();
-        uint8_t* st = smem + stage * kStageStride;
+        uint8_t* st = smem + stage * S::kStride;
+        const int kb0 = st_i * j.nslab;   // first K slab of this stage
         if constexpr (kFp8) {
           // weight scale atoms: one scale for the whole 128 x 128 block
-          if (un.down) {
-            const float s0 = __ldg(p.sd + ((int64_t)e * p.n_hslices + un.slice) * (p.I / 128) + kb);
-            const uint32_t w0 = ue8m0_word(s0);
-            reinterpret_cast<uint4*>(st + kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
+          if (down) {
+            const float* sdp = p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * (p.I / 128) + kb0;
+            const uint32_t w0 = ue8m0_word(__ldg(sdp));
+            reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
+            if (j.nslab == 2) {
+              const uint32_t w1 = ue8m0_word(__ldg(sdp + 1));
+              reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
+            }
           } else {
-            const int64_t si = ((int64_t)e * p.n_islices + un.slice) * (p.H / 128) + kb;
+            const int64_t si = ((int64_t)j.e * p.n_islices + j.slice) * (p.H / 128) + kb0;
             const uint32_t w0 = ue8m0_word(__ldg(p.sg + si));
             const uint32_t w1 = ue8m0_word(__ldg(p.su + si));
-            reinterpret_cast<uint4*>(st + kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
-            reinterpret_cast<uint4*>(st + kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
+            reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
+            reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
           }
           ptx::fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(full + stage, tx);
-          const int kx = kb * p.kelems;
-          if (un.down) {
-            ptx::tma_load_2d_hint(st, &p.tm_wd, full + stage, kx, arow, pol);
+          if (down) {
+            for (int s = 0; s < j.nslab; ++s)
+              ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, full + stage, (kb0 + s) * p.kelems, arow, pol);
           } else {
-            ptx::tma_load_2d_hint(st, &p.tm_wg, full + stage, kx, arow, pol);
-            ptx::tma_load_2d_hint(st + kOffA1, &p.tm_wu, full + stage, kx, arow, pol);
+            ptx::tma_load_2d_hint(st, &p.tm_wg, full + stage, kb0 * p.kelems, arow, pol);
+            ptx::tma_load_2d_hint(st + S::kOffA1, &p.tm_wu, full + stage, kb0 * p.kelems, arow, pol);
           }
-          const void* tmb = un.down ? (const void*)&p.tm_h : (const void*)&p.tm_x;
-          for (int j = 0; j < N / 16; ++j) ptx::tma_load_2d(st + kOffB + j * 2048, tmb, full + stage, kx, row0 + 16 * j);
+          const void* tmb = down ? (const void*)&p.tm_h : (const void*)&p.tm_x;
+          for (int s = 0; s < j.nslab; ++s)
+            for (int r = 0; r < N / 16; ++r)
+              ptx::tma_load_2d(st + S::kOffB + s * N * kSlab + r * 2048, tmb, full + stage, (kb0 + s) * p.kelems,
+                               brow + 16 * r);
           if constexpr (kFp8) {
-            const uint8_t* sf = un.down ? p.ws.hsf + (tile_g * (p.I / 128) + kb) * kSfAtomBytes
-                                        : p.ws.xsf + (tile_g * (p.H / 128) + kb) * kSfAtomBytes;
-            ptx::bulk_load(st + kOffSfb, sf, kSfAtomBytes, full + stage);
+            for (int s = 0; s < j.nslab; ++s) {
+              const uint8_t* sf = down ? p.ws.hsf + (tile_g * (p.I / 128) + kb0 + s) * kSfAtomBytes
+                                       : p.ws.xsf + (tile_g * (p.H / 128) + kb0 + s) * kSfAtomBytes;
+              ptx::bulk_load(st + S::kOffSfb0 + s * kSfAtomBytes, sf, kSfAtomBytes, full + stage);
+            }
           }
         }
         __syncwarp();
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
       }
+      if (!ok) break;
     }
     // drain: every load this warp started has landed before the CTA exits
     if (lane == 0) {
@@ -306,63 +412,99 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    uint32_t stage = 0, phase = 0, acc_phase = 0;
-    bool ok = true;
-    for (uint32_t u = blockIdx.x; ok && u < total; u += gridDim.x) {
-      const Unit un = unit_of(u, n1, p.n_islices, p.n_hslices);
-      int rows = 0, good = 1;
+    // Two 128-column accumulator slots: a job with N <= 64 (or a down job)
+    // takes one (gate at +0, up at +64), a gate/up job with N > 64 takes both,
+    // so the next job's MMAs overlap the previous job's epilogue.
+    uint32_t stage = 0, phase = 0, acc_ph = 0 /* bit per slot */, next_slot = 0;
+    for (uint32_t i = 0;; ++i) {
+      int4 raw = make_int4(0, 0, kKindAbort << 16, 0);
       if (lane == 0) {
-        int e, tile;
-        good = fetch_tile(p, epoch, un.slot, abort_flag, &e, &tile, &rows);
-        if (good) good = wait_bar(acc_empty, acc_phase ^ 1u, abort_flag, hdr, 0x50000000u);
+        Job jj;
+        if (take_job(i, &jj)) raw = pack_job(jj);
+      }
+      const Job j = unpack_job(shfl_int4(raw));
+      if (j.kind >= kKindEnd) break;
+      const bool down = j.kind == kKindDown;
+      const int N = (j.rows + 15) & ~15;
+      const bool two = !down && N > 64;
+      const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
+      const uint32_t colG = 128u * s0;
+      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+      int good = 1;
+      if (lane == 0) {
+        good = wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0);
+        if (good && two) good = wait_bar(acc_empty + s1, ((acc_ph >> s1) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s1);
       }
       good = __shfl_sync(0xffffffffu, good, 0);
-      if (!good) { ok = false; break; }
-      rows = __shfl_sync(0xffffffffu, rows, 0);
+      if (!good) break;
       ptx::tc_fence_after();
-      const int N = (rows + 15) & ~15;
-      const int nk = un.down ? p.nk2 : p.nk1;
+      const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
       const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
-      for (int kb = 0; kb < nk; ++kb) {
+      bool ok = true;
+      for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
         if (lane == 0) w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage);
         w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
         if (!w_ok) { ok = false; break; }
         ptx::tc_fence_after();
         if (lane == 0) {
-          uint8_t* st = smem + stage * kStageStride;
+          uint8_t* st = smem + stage * S::kStride;
           if constexpr (kFp8) {
             // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
-            ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + kOffSfa0), 16, 128, ptx::kLayoutNone));
-            if (!un.down)
-              ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + kOffSfa1), 16, 128, ptx::kLayoutNone));
-            ptx::tmem_cp_32x128b_x4(tmem + kColSfb, ptx::smem_desc(ptx::smem_u32(st + kOffSfb), 16, 128, ptx::kLayoutNone));
+            ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
+            ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
+            if (!down || j.nslab == 2)
+              ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
+            if (down && j.nslab == 2)
+              ptx::tmem_cp_32x128b_x4(tmem + kColSfb1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb1), 16, 128, ptx::kLayoutNone));
           }
           const uint64_t a0 = ptx::desc_kmajor_sw128(st);
-          const uint64_t a1 = ptx::desc_kmajor_sw128(st + kOffA1);
-          const uint64_t b = ptx::desc_kmajor_sw128(st + kOffB);
+          const uint64_t a1 = ptx::desc_kmajor_sw128(st + S::kOffA1);
+          const uint64_t b0 = ptx::desc_kmajor_sw128(st + S::kOffB);
+          if (!down) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t off = (uint64_t)(kk * 32) >> 4;   // 32 bytes of K per MMA
-            if constexpr (kFp8) {
-              ptx::mma_mxf8(tmem + kColG, a0 + off, b + off, idesc, tmem + kColSfa0, tmem + kColSfb, acc);
-              if (!un.down)
-                ptx::mma_mxf8(tmem + kColU, a1 + off, b + off, idesc, tmem + kColSfa1, tmem + kColSfb, acc);
-            } else {
-              ptx::mma_f16(tmem + kColG, a0 + off, b + off, idesc, acc);
-              if (!un.down) ptx::mma_f16(tmem + kColU, a1 + off, b + off, idesc, acc);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (st_i > 0 || kk > 0) ? 1u : 0u;
+              const uint64_t off = (uint64_t)(kk * 32) >> 4;   // 32 bytes of K per MMA
+              if constexpr (kFp8) {
+                ptx::mma_mxf8(tmem + colG, a0 + off, b0 + off, idesc, tmem + kColSfa0, tmem + kColSfb0, acc);
+                ptx::mma_mxf8(tmem + colU, a1 + off, b0 + off, idesc, tmem + kColSfa1, tmem + kColSfb0, acc);
+              } else {
+                ptx::mma_f16(tmem + colG, a0 + off, b0 + off, idesc, acc);
+                ptx::mma_f16(tmem + colU, a1 + off, b0 + off, idesc, acc);
+              }
+            }
+          } else {
+            for (int s = 0; s < j.nslab; ++s) {
+              const uint64_t as = s ? a1 : a0;
+              const uint64_t bs = ptx::desc_kmajor_sw128(st + S::kOffB + s * N * kSlab);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (st_i > 0 || s > 0 || kk > 0) ? 1u : 0u;
+                const uint64_t off = (uint64_t)(kk * 32) >> 4;
+                if constexpr (kFp8) {
+                  ptx::mma_mxf8(tmem + colG, as + off, bs + off, idesc, tmem + (s ? kColSfa1 : kColSfa0),
+                                tmem + (s ? kColSfb1 : kColSfb0), acc);
+                } else {
+                  ptx::mma_f16(tmem + colG, as + off, bs + off, idesc, acc);
+                }
+              }
             }
           }
           ptx::mma_commit(empty + stage);   // frees the stage once these MMAs are done
         }
         __syncwarp();
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      if (lane == 0) ptx::mma_commit(acc_full);
+      if (lane == 0) {
+        ptx::mma_commit(acc_full + s0);
+        if (two) ptx::mma_commit(acc_full + s1);
+      }
       __syncwarp();
-      acc_phase ^= 1u;
+      acc_ph ^= 1u << s0;
+      if (two) acc_ph ^= 1u << s1;
+      else next_slot ^= 1u;
     }
     // drain: all MMAs and copies issued by this warp are complete
     if (lane == 0) {
@@ -379,83 +521,102 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     const int f = q * 32 + lane;            // output feature within the slice
     const int et = threadIdx.x - 64;        // 0..127
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    uint32_t acc_phase = 0;
-    for (uint32_t u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit un = unit_of(u, n1, p.n_islices, p.n_hslices);
+    uint32_t acc_ph = 0, next_slot = 0;
+    for (uint32_t i = 0;; ++i) {
       if (et == 0) {
-        int e = 0, tile = 0, rows = 0;
-        int good = fetch_tile(p, epoch, un.slot, abort_flag, &e, &tile, &rows);
-        if (good) good = wait_bar(acc_full, acc_phase, abort_flag, hdr, 0x70000000u);
-        epi_info[0] = good; epi_info[1] = e; epi_info[2] = tile; epi_info[3] = rows;
+        Job jj;
+        int good = take_job(i, &jj);
+        if (!good) jj.kind = kKindAbort;
+        if (jj.kind < kKindEnd) {
+          const int N = (jj.rows + 15) & ~15;
+          const bool two = jj.kind == kKindGateUp && N > 64;
+          const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
+          good = wait_bar(acc_full + s0, (acc_ph >> s0) & 1u, abort_flag, hdr, 0x70000000u | s0);
+          if (good && two) good = wait_bar(acc_full + s1, (acc_ph >> s1) & 1u, abort_flag, hdr, 0x70000000u | s1);
+          if (!good) jj.kind = kKindAbort;
+        }
+        *epi_job = pack_job(jj);
       }
       ptx::named_barrier(1, 128);
-      const int good = epi_info[0], e = epi_info[1], tile = epi_info[2], rows = epi_info[3];
+      const Job j = unpack_job(*epi_job);
       ptx::named_barrier(1, 128);
-      if (!good) break;
-      while (!ptx::mbar_try_wait(acc_full, acc_phase)) {}   // completed: returns at once
+      if (j.kind >= kKindEnd) break;
+      const bool down = j.kind == kKindDown;
+      const int N = (j.rows + 15) & ~15;
+      const bool two = !down && N > 64;
+      const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
+      const uint32_t colG = 128u * s0;
+      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+      while (!ptx::mbar_try_wait(acc_full + s0, (acc_ph >> s0) & 1u)) {}   // completed: returns at once
+      if (two) while (!ptx::mbar_try_wait(acc_full + s1, (acc_ph >> s1) & 1u)) {}
       ptx::tc_fence_after();
-      const int64_t row0 = (int64_t)e * p.cap + (int64_t)tile * kTileRows;
-      const int64_t tile_g = (int64_t)e * p.tpe + tile;
-      for (int n0 = 0; n0 < rows; n0 += 16) {
+      const int64_t row0 = (int64_t)j.e * p.cap + (int64_t)j.tile * kTileRows + j.row_off;
+      const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
+      for (int n0 = 0; n0 < j.rows; n0 += 16) {
         uint32_t g[16], uu[16];
-        ptx::tmem_ld_x16(tmem + lane_base + kColG + n0, g);
-        if (!un.down) ptx::tmem_ld_x16(tmem + lane_base + kColU + n0, uu);
+        ptx::tmem_ld_x16(tmem + lane_base + colG + n0, g);
+        if (!down) ptx::tmem_ld_x16(tmem + lane_base + colU + n0, uu);
         ptx::tmem_wait_ld();
-        const int nv = min(16, rows - n0);
-        if (un.down) {
-          __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(p.y) + (row0 + n0) * p.H + un.slice * 128 + f;
+        const int nv = min(16, j.rows - n0);
+        if (down) {
+          __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(p.y) + (row0 + n0) * p.H + j.slice * 128 + f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < nv) yp[(int64_t)j * p.H] = __float2bfloat16_rn(__uint_as_float(g[j]));
+          for (int jj = 0; jj < 16; ++jj)
+            if (jj < nv) yp[(int64_t)jj * p.H] = __float2bfloat16_rn(__uint_as_float(g[jj]));
           continue;
         }
         float h[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[j] = silu(__uint_as_float(g[j])) * __uint_as_float(uu[j]);
+        for (int jj = 0; jj < 16; ++jj) h[jj] = silu(__uint_as_float(g[jj])) * __uint_as_float(uu[jj]);
         if constexpr (kFp8) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float m = fabsf(h[j]);
+          for (int jj = 0; jj < 16; ++jj) {
+            float m = fabsf(h[jj]);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) red[q * 16 + j] = m;
+            if (lane == 0) red[q * 16 + jj] = m;
           }
           ptx::named_barrier(1, 128);
-          uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + (row0 + n0) * p.I + un.slice * 128 + f;
+          uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float amax = fmaxf(fmaxf(red[j], red[16 + j]), fmaxf(red[32 + j], red[48 + j]));
+          for (int jj = 0; jj < 16; ++jj) {
+            const float amax = fmaxf(fmaxf(red[jj], red[16 + jj]), fmaxf(red[32 + jj], red[48 + jj]));
             const int pe = pow2_scale_exp(amax);
-            if (j < nv) {
-              const uint16_t b2 = cvt_e4m3x2(h[j] * exp2i(-pe > -126 ? -pe : -126), 0.f);
-              hp[(int64_t)j * p.I] = (uint8_t)(b2 & 0xFF);
+            if (jj < nv) {
+              const uint16_t b2 = cvt_e4m3x2(h[jj] * exp2i(-pe > -126 ? -pe : -126), 0.f);
+              hp[(int64_t)jj * p.I] = (uint8_t)(b2 & 0xFF);
               if (f == 0) {
-                const int64_t r = row0 + n0 + j;
-                p.hs[r * (p.I / 128) + un.slice] = exp2i(pe);
-                // scale atom of this tile and slice (row n0 + j of the tile)
-                *reinterpret_cast<uint32_t*>(p.ws.hsf + (tile_g * (p.I / 128) + un.slice) * kSfAtomBytes +
-                                             sf_atom_offset(n0 + j)) = (uint32_t)(pe + 127) * 0x01010101u;
+                const int64_t r = row0 + n0 + jj;
+                p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
+                // scale atom of this tile and slice (row j.row_off + n0 + jj of the tile)
+                *reinterpret_cast<uint32_t*>(p.ws.hsf + (tile_g * (p.I / 128) + j.slice) * kSfAtomBytes +
+                                             sf_atom_offset(j.row_off + n0 + jj)) = (uint32_t)(pe + 127) * 0x01010101u;
               }
             }
           }
           ptx::named_barrier(1, 128);     // red[] is reused by the next chunk
         } else {
-          __nv_bfloat16* hp = reinterpret_cast<__nv_bfloat16*>(p.hq) + (row0 + n0) * p.I + un.slice * 128 + f;
+          __nv_bfloat16* hp = reinterpret_cast<__nv_bfloat16*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < nv) hp[(int64_t)j * p.I] = __float2bfloat16_rn(h[j]);
+          for (int jj = 0; jj < 16; ++jj)
+            if (jj < nv) hp[(int64_t)jj * p.I] = __float2bfloat16_rn(h[jj]);
         }
       }
-      // accumulators consumed: let the MMA warp start the next unit
+      // accumulators consumed: let the MMA warp reuse the slot(s)
       ptx::tc_fence_before();
       ptx::named_barrier(1, 128);
-      if (et == 0) ptx::mbar_arrive(acc_empty);
-      acc_phase ^= 1u;
-      if (!un.down) {
-        // publish this slice of h to the down units of the same tile
+      if (et == 0) {
+        ptx::mbar_arrive(acc_empty + s0);
+        if (two) ptx::mbar_arrive(acc_empty + s1);
+      }
+      acc_ph ^= 1u << s0;
+      if (two) acc_ph ^= 1u << s1;
+      else next_slot ^= 1u;
+      if (!down) {
+        // publish this chunk of this slice of h to the down jobs of the tile
         __threadfence();
         ptx::named_barrier(1, 128);
-        if (et == 0) atomicAdd(hdone + un.slot, 1u);
+        if (et == 0) atomicAdd(hdone + j.slot, 1u);
       }
     }
   }
@@ -465,6 +626,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA out records that one more FFN call ran on this dispatch
+    __threadfence();
+    const uint32_t exits = atomicAdd(misc + kFfnExit, 1u) + 1u;
+    if (exits == gridDim.x * (gen + 1u)) st_release(misc + kFfnGen, gen + 1u);
   }
 }
 
@@ -500,12 +667,14 @@ bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int64_t cols, int64_t
   return r == CUDA_SUCCESS;
 }
 
-template <bool kFp8>
+template <bool kFp8, int kBRows>
 cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
+  using S = Stage<kBRows>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(ffn_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    attr_err = cudaFuncSetAttribute(ffn_tc_kernel<kFp8, kBRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    S::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   TcParams p;
@@ -536,8 +705,19 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.nk1 = (int)(H / kel);
   p.nk2 = (int)(I / kel);
   p.tiles = c.L.tiles;
-  ffn_tc_kernel<kFp8><<<c.num_sms, kThreads, kSmemBytes, c.stream>>>(p);
+  ffn_tc_kernel<kFp8, kBRows><<<c.num_sms, kThreads, S::kSmemBytes, c.stream>>>(p);
   return cudaGetLastError();
+}
+
+// Token tiles of up to 64 rows give a deeper pipeline (5 stages instead of 4);
+// they suit layers whose experts see few tokens each (decode). Bigger tiles are
+// split into 64-row chunks, which re-streams their weights, so layers with
+// many tokens per expert use 128-row tiles.
+template <bool kFp8>
+cudaError_t launch_by_rows(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
+  const int64_t rows_per_expert = c.s.T * c.s.topk / c.s.E;
+  if (rows_per_expert <= 32) return launch_typed<kFp8, 64>(c, b, w, y);
+  return launch_typed<kFp8, 128>(c, b, w, y);
 }
 
 }  // namespace
@@ -552,7 +732,7 @@ bool ffn_tc_supported(const moe_shape& s) {
 }
 
 cudaError_t launch_ffn_tc(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
-  return c.s.weight_dtype == MOE_E4M3 ? launch_typed<true>(c, b, w, y) : launch_typed<false>(c, b, w, y);
+  return c.s.weight_dtype == MOE_E4M3 ? launch_by_rows<true>(c, b, w, y) : launch_by_rows<false>(c, b, w, y);
 }
 
 }  // namespace moe
