@@ -32,7 +32,7 @@ PROFILES = os.path.join(ROOT, "profiles")
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--config", default="decode")
     p.add_argument("--T", type=int, default=None, help="override the token count")
@@ -67,56 +67,76 @@ def dist_env():
 # ------------------------------------------------------------ GPU clocks --
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock, its maximum, board power and the active clock
+    event (throttle) reasons of one GPU every few milliseconds through NVML,
+    in a background thread, while the timed region runs."""
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.idx = torch_device_index
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.stop_flag = False
+        self.nvml = None
+        self.handle = None
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        try:
+            props = torch.cuda.get_device_properties(self.idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _run(self):
+        nv, h = self.nvml, self.handle
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((sm, mx, pw, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
+        import threading
         try:
-            import tempfile
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self._open()
         except Exception:
-            self.proc = None
+            self.nvml = None
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.rows and time.time() - t0 < 1.0:
+            time.sleep(0.001)
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        if not self.rows:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = set()
-        for r in rows:
-            for n, v in zip(names, r[3][1:]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows)}
+        for r in self.rows:
+            for bit, name in self.REASONS.items():
+                if r[3] & bit:
+                    reasons.add(name)
+        loaded = [r[0] for r in self.rows if r[2] > 200.0] or [r[0] for r in self.rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": sorted(reasons), "samples": len(self.rows),
+                "power_w_max": max(r[2] for r in self.rows), "source": "NVML, 2 ms period"}
 
 
 # ------------------------------------------------------------ CPU oracle --

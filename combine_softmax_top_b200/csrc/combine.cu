@@ -7,16 +7,21 @@
 //
 //   out[t] = sum_{j < k} w[t, j] * y[pos[t*k + j]]    (fp32, slot order)
 //
-// rounded once to the output dtype. Grid (H chunks, tokens): each thread owns
-// 8 consecutive outputs and issues the k gathers (16-byte loads for bf16 / 8
-// for e4m3) before the FMAs so the loads overlap.
+// rounded once to the output dtype. Work unit = (token, 512-value chunk of
+// the row); each warp walks units grid-stride. Lanes j < k load pos/w of the
+// token and broadcast them; every lane then owns 16 consecutive outputs and
+// issues the k row loads (32 bytes each for bf16, 16 for e4m3) before any
+// arithmetic, so a warp keeps k x 1 KB in flight per unit.
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kVec = 8;  // outputs per thread
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kVec = 16;                 // outputs per lane per unit
+constexpr int kChunk = 32 * kVec;        // outputs per unit
+constexpr int kBatch = 8;                // slots loaded together
 
 struct Args {
   const int32_t* pos;
@@ -25,74 +30,114 @@ struct Args {
   const float* xs;    // e4m3 identity rows: scales
   void* out;
   int T, H, k;
-  int row_dtype;      // MOE_F32 / MOE_BF16 / MOE_E4M3
-  int out_dtype;
 };
 
-__device__ __forceinline__ void load_row8(const Args& a, int row, int h0, float* v) {
+// Raw bytes of 16 consecutive values of one row (64 B f32, 32 B bf16, 16 B e4m3).
+template <int kRowDt>
+struct Raw16 {
+  uint4 v[kRowDt == MOE_F32 ? 4 : (kRowDt == MOE_BF16 ? 2 : 1)];
+};
+
+template <int kRowDt>
+__device__ __forceinline__ void load_raw(const Args& a, int row, int h0, Raw16<kRowDt>& r, float& s) {
   const int64_t off = (int64_t)row * a.H + h0;
-  if (a.row_dtype == MOE_BF16) {
-    uint4 q = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.rows) + off));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  if constexpr (kRowDt == MOE_BF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.rows) + off);
+    r.v[0] = __ldg(p);
+    r.v[1] = __ldg(p + 1);
+  } else if constexpr (kRowDt == MOE_F32) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(a.rows) + off);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  } else if (a.row_dtype == MOE_F32) {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.rows) + off);
-    float4 q0 = __ldg(p), q1 = __ldg(p + 1);
-    v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
-    v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+    for (int i = 0; i < 4; ++i) r.v[i] = __ldg(p + i);
   } else {
-    uint2 q = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(a.rows) + off));
-    const float s = __ldg(a.xs + (int64_t)row * (a.H / kQBlock) + h0 / kQBlock);
-    const uint32_t w[2] = {q.x, q.y};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = e4m3_to_f32((uint8_t)(w[i / 4] >> (8 * (i % 4)))) * s;
+    r.v[0] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.rows) + off));
+    s = __ldg(a.xs + (int64_t)row * (a.H / kQBlock) + h0 / kQBlock);
   }
 }
 
-__global__ void __launch_bounds__(kThreads) combine_kernel(Args a) {
-  const int t = blockIdx.y;
-  const int h0 = (blockIdx.x * kThreads + threadIdx.x) * kVec;
-  if (h0 >= a.H) return;
-  float acc[kVec];
+template <int kRowDt>
+__device__ __forceinline__ void fma_raw(const Raw16<kRowDt>& r, float s, float wj, float* acc) {
+  if constexpr (kRowDt == MOE_BF16) {
+    const uint32_t u[8] = {r.v[0].x, r.v[0].y, r.v[0].z, r.v[0].w, r.v[1].x, r.v[1].y, r.v[1].z, r.v[1].w};
 #pragma unroll
-  for (int i = 0; i < kVec; ++i) acc[i] = 0.f;
-  constexpr int kBatch = 8;  // gathers in flight per thread
-  for (int j0 = 0; j0 < a.k; j0 += kBatch) {
-    float v[kBatch][kVec];
-    float wj[kBatch];
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int j = j0 + b;
-      const int row = j < a.k ? __ldg(a.pos + (int64_t)t * a.k + j) : -1;
-      wj[b] = row >= 0 ? __ldg(a.w + (int64_t)t * a.k + j) : 0.f;
-      if (row >= 0) load_row8(a, row, h0, v[b]);
-      else {
-#pragma unroll
-        for (int i = 0; i < kVec; ++i) v[b][i] = 0.f;
-      }
+    for (int i = 0; i < 8; ++i) {
+      acc[2 * i] = fmaf(wj, __uint_as_float(u[i] << 16), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wj, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
     }
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b)
-#pragma unroll
-      for (int i = 0; i < kVec; ++i) acc[i] = fmaf(wj[b], v[b][i], acc[i]);
-  }
-  const int64_t off = (int64_t)t * a.H + h0;
-  if (a.out_dtype == MOE_BF16) {
-    uint32_t w[4];
+  } else if constexpr (kRowDt == MOE_F32) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&b2);
+      acc[4 * i] = fmaf(wj, __uint_as_float(r.v[i].x), acc[4 * i]);
+      acc[4 * i + 1] = fmaf(wj, __uint_as_float(r.v[i].y), acc[4 * i + 1]);
+      acc[4 * i + 2] = fmaf(wj, __uint_as_float(r.v[i].z), acc[4 * i + 2]);
+      acc[4 * i + 3] = fmaf(wj, __uint_as_float(r.v[i].w), acc[4 * i + 3]);
     }
-    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + off) = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
-    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + off);
-    p[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    p[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    const uint32_t u[4] = {r.v[0].x, r.v[0].y, r.v[0].z, r.v[0].w};
+    const float ws = wj * s;   // w_j * scale: exact scaling by a power of two
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(u[i / 2] >> (16 * (i % 2))), __NV_E4M3);
+      const float2 f2 = __half22float2(__half2(h2));
+      acc[2 * i] = fmaf(ws, f2.x, acc[2 * i]);
+      acc[2 * i + 1] = fmaf(ws, f2.y, acc[2 * i + 1]);
+    }
+  }
+}
+
+template <int kRowDt, int kOutDt>
+__global__ void __launch_bounds__(kThreads) combine_kernel(Args a) {
+  const int lane = threadIdx.x & 31;
+  const int nch = (a.H + kChunk - 1) / kChunk;
+  const int64_t units = (int64_t)a.T * nch;
+  const int64_t nw = (int64_t)gridDim.x * kWarps;
+  for (int64_t u = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); u < units; u += nw) {
+    const int t = (int)(u / nch);
+    const int h0 = (int)(u % nch) * kChunk + lane * kVec;
+    const bool live = h0 < a.H;
+    float acc[kVec];
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) acc[i] = 0.f;
+    for (int j0 = 0; j0 < a.k; j0 += 32) {
+      // lanes j < k hold pos / w of slot j0 + j
+      const int jl = j0 + lane;
+      const int my_row = jl < a.k ? __ldg(a.pos + (int64_t)t * a.k + jl) : -1;
+      const float my_w = jl < a.k ? __ldg(a.w + (int64_t)t * a.k + jl) : 0.f;
+      const int nj = min(32, a.k - j0);
+      for (int b0 = 0; b0 < nj; b0 += kBatch) {
+        Raw16<kRowDt> r[kBatch];
+        float sc[kBatch];
+        float wj[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int row = __shfl_sync(0xffffffffu, my_row, (b0 + b) & 31);
+          wj[b] = __shfl_sync(0xffffffffu, my_w, (b0 + b) & 31);
+          sc[b] = 0.f;
+          if (b0 + b < nj && row >= 0 && live) load_raw<kRowDt>(a, row, h0, r[b], sc[b]);
+          else wj[b] = 0.f;
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b)
+          if (wj[b] != 0.f) fma_raw<kRowDt>(r[b], sc[b], wj[b], acc);
+      }
+    }
+    if (!live) continue;
+    const int64_t off = (int64_t)t * a.H + h0;
+    if constexpr (kOutDt == MOE_BF16) {
+      uint32_t wv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        wv[i] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + off);
+      p[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      p[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+    } else {
+      float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + off);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+    }
   }
 }
 
@@ -107,19 +152,31 @@ cudaError_t launch_combine(const Ctx& c, const moe_dispatch_bufs& b, const void*
   a.H = (int)c.s.H;
   a.k = (int)c.s.topk;
   a.out = out;
-  a.out_dtype = c.s.out_dtype;
+  int row_dt;
   if (c.s.identity_experts) {
     a.rows = b.xq;
     a.xs = b.xs;
-    a.row_dtype = c.s.xq_dtype;
+    row_dt = c.s.xq_dtype;
   } else {
     a.rows = y;
     a.xs = nullptr;
-    a.row_dtype = c.s.y_dtype;
+    row_dt = c.s.y_dtype;
   }
   if (a.T == 0) return cudaSuccess;
-  dim3 grid((unsigned)((a.H + kThreads * kVec - 1) / (kThreads * kVec)), (unsigned)a.T);
-  combine_kernel<<<grid, kThreads, 0, c.stream>>>(a);
+  const int64_t units = (int64_t)a.T * ((a.H + kChunk - 1) / kChunk);
+  const int64_t want = (units + kWarps - 1) / kWarps;
+  const int grid = (int)std::min<int64_t>(want, (int64_t)c.num_sms * 4);
+  const bool bf16_out = c.s.out_dtype == MOE_BF16;
+  if (row_dt == MOE_BF16) {
+    if (bf16_out) combine_kernel<MOE_BF16, MOE_BF16><<<grid, kThreads, 0, c.stream>>>(a);
+    else combine_kernel<MOE_BF16, MOE_F32><<<grid, kThreads, 0, c.stream>>>(a);
+  } else if (row_dt == MOE_F32) {
+    if (bf16_out) combine_kernel<MOE_F32, MOE_BF16><<<grid, kThreads, 0, c.stream>>>(a);
+    else combine_kernel<MOE_F32, MOE_F32><<<grid, kThreads, 0, c.stream>>>(a);
+  } else {
+    if (bf16_out) combine_kernel<MOE_E4M3, MOE_BF16><<<grid, kThreads, 0, c.stream>>>(a);
+    else combine_kernel<MOE_E4M3, MOE_F32><<<grid, kThreads, 0, c.stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -96,6 +96,12 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
 
   const int t = blockIdx.x;
   if (t < a.T) {
+    // the first slice of the row is read before the claims so the load and
+    // the atomics' round trips overlap
+    const int steps = a.H / kElems;
+    float v0[kElems];
+    if (tid < steps) load16(a.x, a.act, (int64_t)t * a.H + tid * kElems, v0);
+
     // 1. claim rows
     if (tid < a.k) {
       const int pair = t * a.k + tid;
@@ -119,13 +125,16 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     __syncthreads();
 
     // 2. stream the row: lane group of 8 covers one 128-value block
-    const int steps = a.H / kElems;
     for (int s = tid; s < (steps + 31) / 32 * 32; s += kThreads) {
       const bool live = s < steps;
       const int h0 = s * kElems;
       float v[kElems];
-      if (live) load16(a.x, a.act, (int64_t)t * a.H + h0, v);
-      else {
+      if (live && s == tid) {
+#pragma unroll
+        for (int i = 0; i < kElems; ++i) v[i] = v0[i];
+      } else if (live) {
+        load16(a.x, a.act, (int64_t)t * a.H + h0, v);
+      } else {
 #pragma unroll
         for (int i = 0; i < kElems; ++i) v[i] = 0.f;
       }

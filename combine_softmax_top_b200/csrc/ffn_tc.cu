@@ -67,7 +67,8 @@ enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
 enum : int { kFfnGen = 3, kFfnExit = 4 };   // counter-set misc slots used here
 
 struct TcParams {
-  CUtensorMap tm_wg, tm_wu, tm_wd, tm_x, tm_h;
+  CUtensorMap tm_wg, tm_wu, tm_wd;
+  CUtensorMap tm_x[4], tm_h[4];   // token rows in boxes of 16, 32, 64, 128 rows
   const float* sg;
   const float* su;
   const float* sd;
@@ -318,8 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ptx::prefetch_tmap(&p.tm_wg);
       ptx::prefetch_tmap(&p.tm_wu);
       ptx::prefetch_tmap(&p.tm_wd);
-      ptx::prefetch_tmap(&p.tm_x);
-      ptx::prefetch_tmap(&p.tm_h);
+      for (int b = 0; b < 4; ++b) {
+        ptx::prefetch_tmap(&p.tm_x[b]);
+        ptx::prefetch_tmap(&p.tm_h[b]);
+      }
     }
     const uint64_t pol = ptx::policy_evict_first();
     uint32_t stage = 0, phase = 0;
@@ -341,6 +344,24 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
       const uint32_t tx = (down ? (uint32_t)j.nslab : 2u) * kABytes + (uint32_t)(j.nslab * N * kSlab) +
                           (kFp8 ? (uint32_t)j.nslab * kSfAtomBytes : 0u);
+      // the job's weight scales, one per 128 x 128 block along K: lane l holds
+      // blocks l and l + 32 (gate/down in sa, up in sb), read once per job
+      uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
+      int sbase = 0;   // first K block held in sa*/sb*
+      const int nkb = down ? p.I / 128 : p.H / 128;
+      const float* pa = down ? p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * nkb
+                             : p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      const float* pb = p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      auto load_scales = [&](int base) {
+        if (lane + base < nkb) sa0 = ue8m0_word(__ldg(pa + base + lane));
+        if (lane + base + 32 < nkb) sa1 = ue8m0_word(__ldg(pa + base + lane + 32));
+        if (!down) {
+          if (lane + base < nkb) sb0 = ue8m0_word(__ldg(pb + base + lane));
+          if (lane + base + 32 < nkb) sb1 = ue8m0_word(__ldg(pb + base + lane + 32));
+        }
+      };
+      if constexpr (kFp8) load_scales(0);
+      const CUtensorMap* tmb = down ? p.tm_h : p.tm_x;   // 16-row boxes
       bool ok = true;
       for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
@@ -352,19 +373,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         const int kb0 = st_i * j.nslab;   // first K slab of this stage
         if constexpr (kFp8) {
           // weight scale atoms: one scale for the whole 128 x 128 block
+          if (kb0 + j.nslab - 1 >= sbase + 64) {   // next 64 blocks of scales (K > 8192)
+            sbase = kb0;
+            load_scales(sbase);
+          }
+          const int kr = kb0 - sbase;
+          const uint32_t w0 = __shfl_sync(0xffffffffu, kr < 32 ? sa0 : sa1, kr & 31);
+          reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
           if (down) {
-            const float* sdp = p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * (p.I / 128) + kb0;
-            const uint32_t w0 = ue8m0_word(__ldg(sdp));
-            reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
             if (j.nslab == 2) {
-              const uint32_t w1 = ue8m0_word(__ldg(sdp + 1));
+              const uint32_t w1 = __shfl_sync(0xffffffffu, kr + 1 < 32 ? sa0 : sa1, (kr + 1) & 31);
               reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
             }
           } else {
-            const int64_t si = ((int64_t)j.e * p.n_islices + j.slice) * (p.H / 128) + kb0;
-            const uint32_t w0 = ue8m0_word(__ldg(p.sg + si));
-            const uint32_t w1 = ue8m0_word(__ldg(p.su + si));
-            reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
+            const uint32_t w1 = __shfl_sync(0xffffffffu, kr < 32 ? sb0 : sb1, kr & 31);
             reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
           }
           ptx::fence_proxy_async_smem();
@@ -379,11 +401,27 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             ptx::tma_load_2d_hint(st, &p.tm_wg, full + stage, kb0 * p.kelems, arow, pol);
             ptx::tma_load_2d_hint(st + S::kOffA1, &p.tm_wu, full + stage, kb0 * p.kelems, arow, pol);
           }
-          const void* tmb = down ? (const void*)&p.tm_h : (const void*)&p.tm_x;
-          for (int s = 0; s < j.nslab; ++s)
-            for (int r = 0; r < N / 16; ++r)
-              ptx::tma_load_2d(st + S::kOffB + s * N * kSlab + r * 2048, tmb, full + stage, (kb0 + s) * p.kelems,
-                               brow + 16 * r);
+          // token rows in the largest boxes that fit: N = 128/64/32/16-row pieces
+          // Small tiles (decode) go in 16-row boxes, large ones in the fewest
+          // boxes of 128/64/32/16 rows; measured, each is the faster choice
+          // for its variant.
+          if constexpr (kBRows <= 64) {
+            for (int s = 0; s < j.nslab; ++s)
+              for (int r = 0; r < N / 16; ++r)
+                ptx::tma_load_2d(st + S::kOffB + s * N * kSlab + r * 2048, tmb, full + stage, (kb0 + s) * p.kelems,
+                                 brow + 16 * r);
+          }
+          for (int s = 0; kBRows > 64 && s < j.nslab; ++s) {
+            uint8_t* dst = st + S::kOffB + s * N * kSlab;
+            const int kx = (kb0 + s) * p.kelems;
+            {
+              int r = 0;
+              if (N - r >= 128) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[3] : &p.tm_x[3], full + stage, kx, brow + r); r += 128; }
+              if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[2] : &p.tm_x[2], full + stage, kx, brow + r); r += 64; }
+              if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[1] : &p.tm_x[1], full + stage, kx, brow + r); r += 32; }
+              if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[0] : &p.tm_x[0], full + stage, kx, brow + r); r += 16; }
+            }
+          }
           if constexpr (kFp8) {
             for (int s = 0; s < j.nslab; ++s) {
               const uint8_t* sf = down ? p.ws.hsf + (tile_g * (p.I / 128) + kb0 + s) * kSfAtomBytes
@@ -461,14 +499,17 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           const uint64_t a0 = ptx::desc_kmajor_sw128(st);
           const uint64_t a1 = ptx::desc_kmajor_sw128(st + S::kOffA1);
           const uint64_t b0 = ptx::desc_kmajor_sw128(st + S::kOffB);
+          // the token scale atom covers the whole 128-row tile (row m in TMEM
+          // column m / 32); a chunk starting at row_off reads from column row_off / 32
+          const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
           if (!down) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t acc = (st_i > 0 || kk > 0) ? 1u : 0u;
               const uint64_t off = (uint64_t)(kk * 32) >> 4;   // 32 bytes of K per MMA
               if constexpr (kFp8) {
-                ptx::mma_mxf8(tmem + colG, a0 + off, b0 + off, idesc, tmem + kColSfa0, tmem + kColSfb0, acc);
-                ptx::mma_mxf8(tmem + colU, a1 + off, b0 + off, idesc, tmem + kColSfa1, tmem + kColSfb0, acc);
+                ptx::mma_mxf8(tmem + colG, a0 + off, b0 + off, idesc, tmem + kColSfa0, tmem + kColSfb0 + sfb_off, acc);
+                ptx::mma_mxf8(tmem + colU, a1 + off, b0 + off, idesc, tmem + kColSfa1, tmem + kColSfb0 + sfb_off, acc);
               } else {
                 ptx::mma_f16(tmem + colG, a0 + off, b0 + off, idesc, acc);
                 ptx::mma_f16(tmem + colU, a1 + off, b0 + off, idesc, acc);
@@ -484,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
                 const uint64_t off = (uint64_t)(kk * 32) >> 4;
                 if constexpr (kFp8) {
                   ptx::mma_mxf8(tmem + colG, as + off, bs + off, idesc, tmem + (s ? kColSfa1 : kColSfa0),
-                                tmem + (s ? kColSfb1 : kColSfb0), acc);
+                                tmem + (s ? kColSfb1 : kColSfb0) + sfb_off, acc);
                 } else {
                   ptx::mma_f16(tmem + colG, as + off, bs + off, idesc, acc);
                 }
@@ -683,10 +724,13 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   const int kel = kFp8 ? 128 : 64;
   if (!make_tmap(&p.tm_wg, w.w_gate, kFp8, H, E * I, kel, 128) ||
       !make_tmap(&p.tm_wu, w.w_up, kFp8, H, E * I, kel, 128) ||
-      !make_tmap(&p.tm_wd, w.w_down, kFp8, I, E * H, kel, 128) ||
-      !make_tmap(&p.tm_x, b.xq, kFp8, H, rows, kel, 16) ||
-      !make_tmap(&p.tm_h, b.hq, kFp8, I, rows, kel, 16))
+      !make_tmap(&p.tm_wd, w.w_down, kFp8, I, E * H, kel, 128))
     return cudaErrorInvalidValue;
+  for (int bx = 0; bx < 4; ++bx) {
+    if (!make_tmap(&p.tm_x[bx], b.xq, kFp8, H, rows, kel, 16 << bx) ||
+        !make_tmap(&p.tm_h[bx], b.hq, kFp8, I, rows, kel, 16 << bx))
+      return cudaErrorInvalidValue;
+  }
   p.sg = w.s_gate;
   p.su = w.s_up;
   p.sd = w.s_down;

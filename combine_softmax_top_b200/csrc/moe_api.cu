@@ -74,7 +74,8 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_h) {
   if (!b) return MOE_ERR_INVALID_ARG;
-  if (!b->xq || !b->counts || !b->offsets || !b->row_src || !b->pos) return MOE_ERR_INVALID_ARG;
+  if (!b->xq || !b->counts || !b->offsets || !b->row_src) return MOE_ERR_INVALID_ARG;
+  if (!b->pos && s->T > 0) return MOE_ERR_INVALID_ARG;   // [T*topk]: may be NULL when T == 0
   if (!aligned16(b->xq)) return MOE_ERR_INVALID_ARG;
   if (s->xq_dtype == MOE_E4M3 && (!b->xs || !aligned16(b->xs))) return MOE_ERR_INVALID_ARG;
   if (need_h && !s->identity_experts) {
@@ -99,13 +100,16 @@ __global__ void init_ws_kernel(uint32_t* words, size_t n) {
   if (blockIdx.x == 0 && threadIdx.x == 0) words[0] = 1u;   // Header::epoch_next
 }
 
+// Token-sized arrays may be NULL when there are no tokens.
+bool tok_ok(const Ctx& c, const void* p) { return c.s.T == 0 || p != nullptr; }
+
 moe_status do_route(const Ctx& c, const float* logits, int32_t* idx, float* w) {
-  if (!logits || !idx || !w || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  if (!tok_ok(c, logits) || !tok_ok(c, idx) || !tok_ok(c, w) || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_route(c, logits, idx, w));
 }
 
 moe_status do_dispatch(const Ctx& c, const void* x, const int32_t* idx, const moe_dispatch_bufs* b) {
-  if (!x || !idx || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (!tok_ok(c, x) || !tok_ok(c, idx) || !aligned16(x)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_bufs(&c.s, b, false);
   if (st != MOE_OK) return st;
   return cuda_status(launch_dispatch(c, x, idx, *b));
@@ -124,7 +128,8 @@ moe_status do_ffn(const Ctx& c, const moe_dispatch_bufs* b, const moe_weights* w
 
 moe_status do_combine(const Ctx& c, const moe_dispatch_bufs* b, const void* y, const float* topk_w,
                       void* out) {
-  if (!b || !b->pos || !topk_w || !out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (!b || !tok_ok(c, b->pos) || !tok_ok(c, topk_w) || !tok_ok(c, out) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
   if (c.s.identity_experts) {
     if (!b->xq || !aligned16(b->xq)) return MOE_ERR_INVALID_ARG;
     if (c.s.xq_dtype == MOE_E4M3 && !b->xs) return MOE_ERR_INVALID_ARG;
@@ -196,8 +201,8 @@ moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits,
   moe_status st = make_ctx(shape, ws, stream, &c);
   if (st != MOE_OK) return st;
   // every argument is checked before the first launch
-  if (!logits || !topk_idx || !topk_w || !aligned16(logits) || !x || !aligned16(x) || !out ||
-      !aligned16(out))
+  if (!tok_ok(c, logits) || !tok_ok(c, topk_idx) || !tok_ok(c, topk_w) || !aligned16(logits) ||
+      !tok_ok(c, x) || !aligned16(x) || !tok_ok(c, out) || !aligned16(out))
     return MOE_ERR_INVALID_ARG;
   st = check_bufs(shape, bufs, true);
   if (st != MOE_OK) return st;

@@ -6,7 +6,7 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
-#include "../../include/moe.h"
+#include "moe.h"   // include/moe.h (the C ABI)
 
 namespace moe {
 

@@ -34,6 +34,8 @@
  *    and read back by moe_poll_status. The library never traps, aborts or
  *    prints.
  *  - All device buffers must be 16-byte aligned; rows are dense (no padding).
+ *    Arrays sized by T (x, logits, topk_idx, topk_w, pos, out) may be NULL
+ *    when T == 0.
  */
 #ifndef MOE_H_
 #define MOE_H_
