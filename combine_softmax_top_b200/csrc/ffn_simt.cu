@@ -122,15 +122,19 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) { g[i] = 0.f; uu[i] = 0.f; }
       for (int k0 = 0; k0 < K; k0 += kK) {
-        for (int i = tid; i < kR * kK; i += kThreads) {
-          const int r = i / kK, kk = i % kK;
-          float v = 0.f;
+        // every load of this K step is issued before any is used
+        constexpr int kXPer = kR * kK / kThreads;   // 4
+        constexpr int kWPer = kF * kK / kThreads;   // 16
+        float xv[kXPer], wv0[kWPer], wv1[kWPer];
+#pragma unroll
+        for (int i = 0; i < kXPer; ++i) {
+          const int idx = tid + kThreads * i, r = idx / kK, kk = idx % kK;
+          xv[i] = 0.f;
           if (r0 + r < rows) {
             const int64_t row = row0 + r0 + r;
-            v = ld_act(xin, xdt, row * K + k0 + kk);
-            if (xdt == MOE_E4M3) v *= xsc[row * (K / kQBlock) + (k0 + kk) / kQBlock];
+            xv[i] = ld_act(xin, xdt, row * K + k0 + kk);
+            if (xdt == MOE_E4M3) xv[i] *= xsc[row * (K / kQBlock) + (k0 + kk) / kQBlock];
           }
-          sx[r][kk] = v;
         }
         float sc0 = 1.f, sc1 = 1.f;
         if (a.w_dt == MOE_E4M3) {
@@ -138,11 +142,23 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
           sc0 = s0[sidx];
           if (!DOWN) sc1 = s1[sidx];
         }
-        for (int i = tid; i < kF * kK; i += kThreads) {
-          const int ff = i / kK, kk = i % kK;
+#pragma unroll
+        for (int i = 0; i < kWPer; ++i) {
+          const int idx = tid + kThreads * i, ff = idx / kK, kk = idx % kK;
           const int64_t widx = (wrow0 + ff) * K + k0 + kk;
-          sw0[ff][kk] = ld_act(w0, a.w_dt, widx) * sc0;
-          if (!DOWN) sw1[ff][kk] = ld_act(w1, a.w_dt, widx) * sc1;
+          wv0[i] = ld_act(w0, a.w_dt, widx);
+          wv1[i] = DOWN ? 0.f : ld_act(w1, a.w_dt, widx);
+        }
+#pragma unroll
+        for (int i = 0; i < kXPer; ++i) {
+          const int idx = tid + kThreads * i;
+          sx[idx / kK][idx % kK] = xv[i];
+        }
+#pragma unroll
+        for (int i = 0; i < kWPer; ++i) {
+          const int idx = tid + kThreads * i;
+          sw0[idx / kK][idx % kK] = wv0[i] * sc0;
+          if (!DOWN) sw1[idx / kK][idx % kK] = wv1[i] * sc1;
         }
         __syncthreads();
 #pragma unroll 4

@@ -41,6 +41,7 @@ constexpr int kSlab = 128;      // K bytes per slab (one 128-byte swizzle row)
 constexpr int kABytes = 128 * kSlab;   // 128 weight rows of one slab
 constexpr int kMaxDynSmem = 232448;    // 227 KB per CTA
 constexpr int kCtlBytes = 1024;        // barriers, unit queue, flags, reductions (664 B used)
+constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert first-tile table (E <= 1024)
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
 // A0 | A1 | B (kBRows x 128 B, or two slabs of N rows) | SFA0 | SFA1 | SFB0 | SFB1
@@ -53,9 +54,9 @@ struct Stage {
   static constexpr int kOffSfb0 = kOffSfa1 + kSfAtomBytes;
   static constexpr int kOffSfb1 = kOffSfb0 + kSfAtomBytes;
   static constexpr int kStride = (kOffSfb1 + kSfAtomBytes + 1023) / 1024 * 1024;
-  static constexpr int kStages = (kMaxDynSmem - kCtlBytes - 1024) / kStride;
+  static constexpr int kStages = (kMaxDynSmem - kCtlBytes - kTileTabBytes - 1024) / kStride;
   static constexpr int kBarOffset = kStages * kStride;
-  static constexpr int kSmemBytes = kBarOffset + kCtlBytes + 1024 /* alignment slack */;
+  static constexpr int kSmemBytes = kBarOffset + kCtlBytes + kTileTabBytes + 1024 /* alignment slack */;
   static_assert(kStages >= 3, "pipeline depth");
 };
 
@@ -131,36 +132,17 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_fla
   }
 }
 
-// The tile behind ring slot `slot` of this epoch: expert, tile index, rows.
-__device__ bool fetch_tile(const TcParams& p, uint32_t epoch, uint32_t slot, volatile int* abort_flag,
-                           int* e, int* tile, int* rows) {
+// Rows of tile `tile` of expert `e` once its sentinel carries this epoch.
+__device__ bool wait_tile(const TcParams& p, uint32_t epoch, int e, int tile, volatile int* abort_flag,
+                          int* rows) {
   const unsigned long long t0 = globaltimer();
-  unsigned long long ent;
-  while (true) {
-    ent = ld_acquire64(p.ws.ring + slot);
-    if ((uint32_t)(ent >> 32) == epoch) break;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitBudgetNs) {
-      latch_error(p.ws.hdr, MOE_ERR_TIMEOUT, 0x10000000u | slot);
-      *abort_flag = 1;
-      return false;
-    }
-    __nanosleep(128);
-  }
-  *e = (int)((ent >> 16) & 0xFFFF);
-  *tile = (int)(ent & 0xFFFF);
-  if (*e >= p.E || *tile >= p.tpe) {          // never published: a corrupt workspace
-    latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x11000000u | slot);
-    *abort_flag = 1;
-    return false;
-  }
-  const uint32_t* sp = p.ws.sentinel + (int64_t)(*e) * p.tpe + *tile;
+  const uint32_t* sp = p.ws.sentinel + (int64_t)e * p.tpe + tile;
   while (true) {
     const uint32_t s = ld_acquire(sp);
     if ((s >> 8) == (epoch & 0xFFFFFFu)) {
       *rows = (int)(s & 0xFF);
       if (*rows < 1 || *rows > kTileRows) {   // never published: a corrupt workspace
-        latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x21000000u | slot);
+        latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x22000000u | (uint32_t)(e * p.tpe + tile));
         *abort_flag = 1;
         return false;
       }
@@ -168,7 +150,7 @@ __device__ bool fetch_tile(const TcParams& p, uint32_t epoch, uint32_t slot, vol
     }
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitBudgetNs) {
-      latch_error(p.ws.hdr, MOE_ERR_TIMEOUT, 0x20000000u | slot);
+      latch_error(p.ws.hdr, MOE_ERR_TIMEOUT, 0x23000000u | (uint32_t)(e * p.tpe + tile));
       *abort_flag = 1;
       return false;
     }
@@ -269,10 +251,38 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
 
   if (warp == 6) {
     // ---------------------------------------------------------------- scheduler
-    // Units (ring slot x 128-feature slice; all gate/up units before all down
-    // units) are dealt round-robin to the CTAs. For each unit the scheduler
-    // resolves the tile (ring entry + sentinel), waits for a down unit's h,
-    // splits the tile into chunks of <= kBRows rows and queues them.
+    // Units, expert-major: for each expert, for each 128-feature slice, every
+    // tile of that expert (all gate/up units before all down units), dealt
+    // round-robin to the CTAs. Neighbouring CTAs thus work on the tiles of one
+    // expert with the same weight slice at the same time and share it in L2.
+    // For each unit the scheduler waits for the tile's sentinel (and a down
+    // unit's h), splits the tile into chunks of <= kBRows rows and queues them.
+    int* tile_pre = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1] first tile of each expert
+    {
+      const uint32_t* cnt = set_count(set);
+      const int per = (p.E + 31) / 32;
+      int local = 0;
+      for (int i = 0; i < per; ++i) {
+        const int e = lane * per + i;
+        if (e < p.E) local += ((int)min(ld_acquire(cnt + e), (uint32_t)p.cap) + kTileRows - 1) / kTileRows;
+      }
+      int incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      int run = incl - local;
+      for (int i = 0; i < per; ++i) {
+        const int e = lane * per + i;
+        if (e < p.E) {
+          tile_pre[e] = run;
+          run += ((int)min(ld_acquire(cnt + e), (uint32_t)p.cap) + kTileRows - 1) / kTileRows;
+        }
+      }
+      if (lane == 31) tile_pre[p.E] = incl;
+      __syncwarp();
+    }
     if (lane == 0) {
       uint32_t i = 0;
       bool good = true;
@@ -284,15 +294,32 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         ++i;
         return true;
       };
+      const uint32_t ntab = (uint32_t)tile_pre[p.E];
+      if (ntab != ntiles) {   // the published tile total disagrees with the counts
+        latch_error(hdr, MOE_ERR_INVALID_ARG, 0x24000000u | ntab);
+        *abort_flag = 1;
+        good = false;
+      }
       for (uint32_t u = blockIdx.x; good && u < total; u += gridDim.x) {
         Job j;
         j.kind = u >= n1 ? kKindDown : kKindGateUp;
         const uint32_t v = j.kind == kKindDown ? u - n1 : u;
-        const int ns = j.kind == kKindDown ? p.n_hslices : p.n_islices;
-        j.slot = (int)(v / ns);
-        j.slice = (int)(v % ns);
+        const uint32_t ns = (uint32_t)(j.kind == kKindDown ? p.n_hslices : p.n_islices);
+        // expert: the last e with tile_pre[e] * ns <= v (empty experts never are)
+        int lo = 0, hi = p.E - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if ((uint32_t)tile_pre[mid] * ns <= v) lo = mid;
+          else hi = mid - 1;
+        }
+        j.e = lo;
+        const uint32_t nt = (uint32_t)(tile_pre[lo + 1] - tile_pre[lo]);
+        const uint32_t w = v - (uint32_t)tile_pre[lo] * ns;
+        j.slice = (int)(w / nt);
+        j.tile = (int)(w % nt);
+        j.slot = j.e * p.tpe + j.tile;     // global tile id: the down units' counter
         int rows = 0;
-        good = fetch_tile(p, epoch, (uint32_t)j.slot, abort_flag, &j.e, &j.tile, &rows);
+        good = wait_tile(p, epoch, j.e, j.tile, abort_flag, &rows);
         if (!good) break;
         const int nch = (rows + kBRows - 1) / kBRows;
         if (j.kind == kKindDown)

@@ -244,7 +244,7 @@ def test_identity_experts_return_input(T, cuda_device):
 # ------------------------------------------------------- bounded waits --
 
 def test_ffn_wait_runs_out_and_context_survives(cuda_device):
-    """Announce one more tile than dispatch published: the FFN's wait for it
+    """Withdraw one published tile's sentinel: the FFN's wait for that tile
     must give up (MOE_ERR_TIMEOUT) instead of hanging, and the device must
     stay usable."""
     s = W.spec("decode", T=32, H=512, E=16, k=4, I=256)
@@ -253,15 +253,17 @@ def test_ffn_wait_runs_out_and_context_survives(cuda_device):
     moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws)
     moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, b.dispatch_bufs())
     assert G.poll(b) == 0
-    # workspace layout: 256-byte header (epoch_next, epoch_cur, ...), then the
-    # counter sets; after the first dispatch epoch_cur = 1 -> set 1, whose
-    # third word is the published tile total
+    # workspace layout: 256-byte header (epoch_next, epoch_cur, ...), two
+    # counter sets, then one 32-bit sentinel per (expert, 128-row tile)
     hdr = b.ws[:16].view(torch.int32)
     assert int(hdr[1]) == 1
-    set_words = 8 + s.E + 2 * s.E * (s.cap // 128)
-    set1 = 256 + ((set_words * 4 + 255) // 256) * 256
-    total = b.ws[set1 + 8:set1 + 12].view(torch.int32)
-    total += 1                                   # a tile nothing will ever publish
+    tpe = s.cap // 128
+    set_words = 8 + s.E + 2 * s.E * tpe
+    sent_off = 256 + 2 * (((set_words * 4 + 255) // 256) * 256)
+    sentinels = b.ws[sent_off:sent_off + 4 * s.E * tpe].view(torch.int32)
+    e = int(np.nonzero(b.counts.cpu().numpy())[0][0])
+    assert int(sentinels[e * tpe]) >> 8 == 1     # published in epoch 1
+    sentinels[e * tpe] = 0                       # as if never published
     torch.cuda.synchronize()
     moe.moe_grouped_ffn(b.shape, b.dispatch_bufs(), moe.weights_struct(inp), b.ws, b.y)
     assert G.poll(b) == 5                        # MOE_ERR_TIMEOUT
