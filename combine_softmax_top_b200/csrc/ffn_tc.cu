@@ -40,7 +40,7 @@ constexpr int kUQ = 8;          // unit-queue depth
 constexpr int kSlab = 128;      // K bytes per slab (one 128-byte swizzle row)
 constexpr int kABytes = 128 * kSlab;   // 128 weight rows of one slab
 constexpr int kMaxDynSmem = 232448;    // 227 KB per CTA
-constexpr int kCtlBytes = 1024;        // barriers, unit queue, flags, reductions (664 B used)
+constexpr int kCtlBytes = 1024;        // barriers, job queue, flags, reductions
 constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert first-tile table (E <= 1024)
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
@@ -174,7 +174,7 @@ __device__ bool wait_count(const uint32_t* count, uint32_t target, volatile int*
   return true;
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.f + expf(-g)); }
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.f + expf(-g)); }
 
 __device__ __forceinline__ uint32_t ue8m0_word(float s) {
   return ((__float_as_uint(s) >> 23) & 0xFFu) * 0x01010101u;
@@ -196,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   uint64_t* uq_empty = uq_full + kUQ;         // [kUQ]
   static_assert((2 * kStages + 5 + 2 * kUQ) * 8 <= 256, "barriers fit before the job queue");
   int4* uq = reinterpret_cast<int4*>(ctl + 256);               // [kUQ] packed jobs
-  float* red = reinterpret_cast<float*>(ctl + 384);            // [4 warps][16 tokens]
-  int4* epi_job = reinterpret_cast<int4*>(ctl + 640);          // job broadcast to the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 656);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 660);
+  int4* epi_job = reinterpret_cast<int4*>(ctl + 384);          // job broadcast to the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 400);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 404);
+  float* red = reinterpret_cast<float*>(ctl + 512);            // [4 warps][32 tokens]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -620,53 +620,57 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ptx::tc_fence_after();
       const int64_t row0 = (int64_t)j.e * p.cap + (int64_t)j.tile * kTileRows + j.row_off;
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
-      for (int n0 = 0; n0 < j.rows; n0 += 16) {
-        uint32_t g[16], uu[16];
-        ptx::tmem_ld_x16(tmem + lane_base + colG + n0, g);
-        if (!down) ptx::tmem_ld_x16(tmem + lane_base + colU + n0, uu);
+      // tokens in batches of 32 columns: one TMEM load per operand, the
+      // per-token max over this warp's 32 features in one redux, the max over
+      // the four warps through shared memory
+      for (int n0 = 0; n0 < j.rows; n0 += 32) {
+        uint32_t g[32], uu[32];
+        ptx::tmem_ld_x32(tmem + lane_base + colG + n0, g);
+        if (!down) ptx::tmem_ld_x32(tmem + lane_base + colU + n0, uu);
         ptx::tmem_wait_ld();
-        const int nv = min(16, j.rows - n0);
+        const int nv = min(32, j.rows - n0);
         if (down) {
           __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(p.y) + (row0 + n0) * p.H + j.slice * 128 + f;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
+          for (int jj = 0; jj < 32; ++jj)
             if (jj < nv) yp[(int64_t)jj * p.H] = __float2bfloat16_rn(__uint_as_float(g[jj]));
           continue;
         }
-        float h[16];
+        float h[32];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) h[jj] = silu(__uint_as_float(g[jj])) * __uint_as_float(uu[jj]);
+        for (int jj = 0; jj < 32; ++jj) h[jj] = silu(__uint_as_float(g[jj])) * __uint_as_float(uu[jj]);
         if constexpr (kFp8) {
+          // |h| bit patterns order like the values (non-negative floats)
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            float m = fabsf(h[jj]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) red[q * 16 + jj] = m;
+          for (int jj = 0; jj < 32; ++jj) {
+            const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[jj])));
+            if (lane == jj) red[q * 32 + jj] = __uint_as_float(m);
           }
           ptx::named_barrier(1, 128);
           uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float amax = fmaxf(fmaxf(red[jj], red[16 + jj]), fmaxf(red[32 + jj], red[48 + jj]));
+          for (int jj = 0; jj < 32; ++jj) {
+            const float amax = fmaxf(fmaxf(red[jj], red[32 + jj]), fmaxf(red[64 + jj], red[96 + jj]));
             const int pe = pow2_scale_exp(amax);
             if (jj < nv) {
               const uint16_t b2 = cvt_e4m3x2(h[jj] * exp2i(-pe > -126 ? -pe : -126), 0.f);
               hp[(int64_t)jj * p.I] = (uint8_t)(b2 & 0xFF);
-              if (f == 0) {
-                const int64_t r = row0 + n0 + jj;
-                p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
-                // scale atom of this tile and slice (row j.row_off + n0 + jj of the tile)
-                *reinterpret_cast<uint32_t*>(p.ws.hsf + (tile_g * (p.I / 128) + j.slice) * kSfAtomBytes +
-                                             sf_atom_offset(j.row_off + n0 + jj)) = (uint32_t)(pe + 127) * 0x01010101u;
-              }
             }
           }
-          ptx::named_barrier(1, 128);     // red[] is reused by the next chunk
+          if (f < nv) {   // thread f records token f's scale
+            const float amax = fmaxf(fmaxf(red[f], red[32 + f]), fmaxf(red[64 + f], red[96 + f]));
+            const int pe = pow2_scale_exp(amax);
+            const int64_t r = row0 + n0 + f;
+            p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
+            // scale atom of this tile and slice (row j.row_off + n0 + f of the tile)
+            *reinterpret_cast<uint32_t*>(p.ws.hsf + (tile_g * (p.I / 128) + j.slice) * kSfAtomBytes +
+                                         sf_atom_offset(j.row_off + n0 + f)) = (uint32_t)(pe + 127) * 0x01010101u;
+          }
+          ptx::named_barrier(1, 128);     // red[] is reused by the next batch
         } else {
           __nv_bfloat16* hp = reinterpret_cast<__nv_bfloat16*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
+          for (int jj = 0; jj < 32; ++jj)
             if (jj < nv) hp[(int64_t)jj * p.I] = __float2bfloat16_rn(h[jj]);
         }
       }
