@@ -164,12 +164,9 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
           *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
           if (leader) {
             a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
-            if (a.xsf) {
-              const int tile = row / kTileRows;   // global tile id e * tpe + local (cap % 128 == 0)
-              const int m = row % kTileRows;
-              *reinterpret_cast<uint32_t*>(a.xsf + ((int64_t)tile * (a.H / kQBlock) + blk) * kSfAtomBytes +
-                                           sf_atom_offset(m)) = (uint32_t)(p + 127) * 0x01010101u;
-            }
+            if (a.xsf)   // tile id e * tpe + local = row / 128 since cap % 128 == 0
+              *sf_atom_byte(a.xsf, row / kTileRows, (a.H + 4 * kQBlock - 1) / (4 * kQBlock), blk,
+                            row % kTileRows) = (uint8_t)(p + 127);
           }
         }
       } else if (live) {

@@ -213,9 +213,8 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
             if (f == 0) {
               a.hs[row * (a.I / kQBlock) + slice] = exp2i(p);
               if (a.hsf)
-                *reinterpret_cast<uint32_t*>(a.hsf + ((int64_t)(row / kTileRows) * (a.I / kQBlock) + slice) *
-                                                         kSfAtomBytes + sf_atom_offset((int)(row % kTileRows))) =
-                    (uint32_t)(p + 127) * 0x01010101u;
+                *sf_atom_byte(a.hsf, row / kTileRows, (a.I + 4 * kQBlock - 1) / (4 * kQBlock), slice,
+                              (int)(row % kTileRows)) = (uint8_t)(p + 127);
             }
           }
         }

@@ -44,7 +44,7 @@ constexpr int kCtlBytes = 1024;        // barriers, job queue, flags, reductions
 constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert first-tile table (E <= 1024)
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
-// A0 | A1 | B (kBRows x 128 B, or two slabs of N rows) | SFA0 | SFA1 | SFB0 | SFB1
+// A0 | A1 | B (kBRows x 128 B, or two slabs of N rows) | SFA0 | SFA1 | SFB0
 template <int kBRows>
 struct Stage {
   static constexpr int kOffA1 = kABytes;
@@ -52,8 +52,7 @@ struct Stage {
   static constexpr int kOffSfa0 = kOffB + kBRows * kSlab;
   static constexpr int kOffSfa1 = kOffSfa0 + kSfAtomBytes;
   static constexpr int kOffSfb0 = kOffSfa1 + kSfAtomBytes;
-  static constexpr int kOffSfb1 = kOffSfb0 + kSfAtomBytes;
-  static constexpr int kStride = (kOffSfb1 + kSfAtomBytes + 1023) / 1024 * 1024;
+  static constexpr int kStride = (kOffSfb0 + kSfAtomBytes + 1023) / 1024 * 1024;
   static constexpr int kStages = (kMaxDynSmem - kCtlBytes - kTileTabBytes - 1024) / kStride;
   static constexpr int kBarOffset = kStages * kStride;
   static constexpr int kSmemBytes = kBarOffset + kCtlBytes + kTileTabBytes + 1024 /* alignment slack */;
@@ -62,7 +61,7 @@ struct Stage {
 
 constexpr uint32_t kTmemCols = 512;
 // accumulators: two 128-column slots at columns 0 and 128; scale factors after
-constexpr uint32_t kColSfa0 = 256, kColSfa1 = 260, kColSfb0 = 264, kColSfb1 = 268;
+constexpr uint32_t kColSfa0 = 256, kColSfa1 = 260, kColSfb0 = 264;
 
 enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
 enum : int { kFfnGen = 3, kFfnExit = 4 };   // counter-set misc slots used here
@@ -81,6 +80,7 @@ struct TcParams {
   int n_islices, n_hslices;  // I/128, H/128
   int nk1, nk2;              // K slabs of gate/up (over H) and down (over I)
   int kelems;                // elements per slab
+  int hgroups, igroups;      // scale atoms per tile along H and I (groups of 4 blocks)
   int64_t tiles;
 };
 
@@ -176,9 +176,8 @@ __device__ bool wait_count(const uint32_t* count, uint32_t target, volatile int*
 
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.f + expf(-g)); }
 
-__device__ __forceinline__ uint32_t ue8m0_word(float s) {
-  return ((__float_as_uint(s) >> 23) & 0xFFu) * 0x01010101u;
-}
+// UE8M0 code of a power-of-two fp32 scale: its biased exponent.
+__device__ __forceinline__ uint32_t ue8m0(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
 template <bool kFp8, int kBRows>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -369,10 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int arow = j.e * (down ? p.H : p.I) + j.slice * 128;
       const int brow = j.e * p.cap + j.tile * kTileRows + j.row_off;
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
-      const uint32_t tx = (down ? (uint32_t)j.nslab : 2u) * kABytes + (uint32_t)(j.nslab * N * kSlab) +
-                          (kFp8 ? (uint32_t)j.nslab * kSfAtomBytes : 0u);
+      const uint32_t tx = (down ? (uint32_t)j.nslab : 2u) * kABytes + (uint32_t)(j.nslab * N * kSlab);
       // the job's weight scales, one per 128 x 128 block along K: lane l holds
-      // blocks l and l + 32 (gate/down in sa, up in sb), read once per job
+      // the exponents of blocks l and l + 32 (gate/down in sa, up in sb), read
+      // once per job
       uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
       int sbase = 0;   // first K block held in sa*/sb*
       const int nkb = down ? p.I / 128 : p.H / 128;
@@ -380,12 +379,23 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
                              : p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
       const float* pb = p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
       auto load_scales = [&](int base) {
-        if (lane + base < nkb) sa0 = ue8m0_word(__ldg(pa + base + lane));
-        if (lane + base + 32 < nkb) sa1 = ue8m0_word(__ldg(pa + base + lane + 32));
+        if (lane + base < nkb) sa0 = ue8m0(__ldg(pa + base + lane));
+        if (lane + base + 32 < nkb) sa1 = ue8m0(__ldg(pa + base + lane + 32));
         if (!down) {
-          if (lane + base < nkb) sb0 = ue8m0_word(__ldg(pb + base + lane));
-          if (lane + base + 32 < nkb) sb1 = ue8m0_word(__ldg(pb + base + lane + 32));
+          if (lane + base < nkb) sb0 = ue8m0(__ldg(pb + base + lane));
+          if (lane + base + 32 < nkb) sb1 = ue8m0(__ldg(pb + base + lane + 32));
         }
+      };
+      // the four exponents of blocks kr .. kr+3 (relative to sbase), packed
+      auto pack4 = [&](uint32_t r0, uint32_t r1, int kr) -> uint32_t {
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int kk = kr + b;
+          const uint32_t v = __shfl_sync(0xffffffffu, kk < 32 ? r0 : r1, kk & 31);
+          w |= (kk + sbase < nkb ? v : 0u) << (8 * b);
+        }
+        return w;
       };
       if constexpr (kFp8) load_scales(0);
       const CUtensorMap* tmb = down ? p.tm_h : p.tm_x;   // 16-row boxes
@@ -398,29 +408,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         __syncwarp();
         uint8_t* st = smem + stage * S::kStride;
         const int kb0 = st_i * j.nslab;   // first K slab of this stage
+        // scale atoms cover four K blocks: they travel with the stage that
+        // starts a group of four
+        const bool sf_stage = kFp8 && (kb0 & 3) == 0;
         if constexpr (kFp8) {
-          // weight scale atoms: one scale for the whole 128 x 128 block
-          if (kb0 + j.nslab - 1 >= sbase + 64) {   // next 64 blocks of scales (K > 8192)
-            sbase = kb0;
-            load_scales(sbase);
-          }
-          const int kr = kb0 - sbase;
-          const uint32_t w0 = __shfl_sync(0xffffffffu, kr < 32 ? sa0 : sa1, kr & 31);
-          reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
-          if (down) {
-            if (j.nslab == 2) {
-              const uint32_t w1 = __shfl_sync(0xffffffffu, kr + 1 < 32 ? sa0 : sa1, (kr + 1) & 31);
+          if (sf_stage) {
+            // weight scale atoms: one exponent per 128 x 128 block, the same
+            // for all 128 rows; byte b = block kb0 + b
+            if (kb0 + 3 >= sbase + 64) {   // next 64 blocks of scales (K > 8192)
+              sbase = kb0;
+              load_scales(sbase);
+            }
+            const int kr = kb0 - sbase;
+            const uint32_t w0 = pack4(sa0, sa1, kr);
+            reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
+            if (!down) {
+              const uint32_t w1 = pack4(sb0, sb1, kr);
               reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
             }
-          } else {
-            const uint32_t w1 = __shfl_sync(0xffffffffu, kr < 32 ? sb0 : sb1, kr & 31);
-            reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
+            ptx::fence_proxy_async_smem();
           }
-          ptx::fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(full + stage, tx);
+          ptx::mbar_arrive_expect_tx(full + stage, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
           if (down) {
             for (int s = 0; s < j.nslab; ++s)
               ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, full + stage, (kb0 + s) * p.kelems, arow, pol);
@@ -449,12 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[0] : &p.tm_x[0], full + stage, kx, brow + r); r += 16; }
             }
           }
-          if constexpr (kFp8) {
-            for (int s = 0; s < j.nslab; ++s) {
-              const uint8_t* sf = down ? p.ws.hsf + (tile_g * (p.I / 128) + kb0 + s) * kSfAtomBytes
-                                       : p.ws.xsf + (tile_g * (p.H / 128) + kb0 + s) * kSfAtomBytes;
-              ptx::bulk_load(st + S::kOffSfb0 + s * kSfAtomBytes, sf, kSfAtomBytes, full + stage);
-            }
+          if (sf_stage) {   // the tokens' scale atom of this group of four blocks
+            const uint8_t* sf = down ? p.ws.hsf + (tile_g * p.igroups + kb0 / 4) * kSfAtomBytes
+                                     : p.ws.xsf + (tile_g * p.hgroups + kb0 / 4) * kSfAtomBytes;
+            ptx::bulk_load(st + S::kOffSfb0, sf, kSfAtomBytes, full + stage);
           }
         }
         __syncwarp();
@@ -480,79 +489,79 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // Two 128-column accumulator slots: a job with N <= 64 (or a down job)
     // takes one (gate at +0, up at +64), a gate/up job with N > 64 takes both,
     // so the next job's MMAs overlap the previous job's epilogue.
-    uint32_t stage = 0, phase = 0, acc_ph = 0 /* bit per slot */, next_slot = 0;
-    for (uint32_t i = 0;; ++i) {
-      int4 raw = make_int4(0, 0, kKindAbort << 16, 0);
-      if (lane == 0) {
-        Job jj;
-        if (take_job(i, &jj)) raw = pack_job(jj);
-      }
-      const Job j = unpack_job(shfl_int4(raw));
-      if (j.kind >= kKindEnd) break;
-      const bool down = j.kind == kKindDown;
-      const int N = (j.rows + 15) & ~15;
-      const bool two = !down && N > 64;
-      const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
-      const uint32_t colG = 128u * s0;
-      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
-      int good = 1;
-      if (lane == 0) {
-        good = wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0);
-        if (good && two) good = wait_bar(acc_empty + s1, ((acc_ph >> s1) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s1);
-      }
-      good = __shfl_sync(0xffffffffu, good, 0);
-      if (!good) break;
-      ptx::tc_fence_after();
-      const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
-      const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
-      bool ok = true;
-      for (int st_i = 0; st_i < nsteps; ++st_i) {
-        int w_ok = 1;
-        if (lane == 0) w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage);
-        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-        if (!w_ok) { ok = false; break; }
+    // One thread issues everything (the other lanes wait at the end): no
+    // warp-wide shuffles or syncs per K step.
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, acc_ph = 0 /* bit per slot */, next_slot = 0;
+      for (uint32_t i = 0;; ++i) {
+        Job j;
+        if (!take_job(i, &j) || j.kind >= kKindEnd) break;
+        const bool down = j.kind == kKindDown;
+        const int N = (j.rows + 15) & ~15;
+        const bool two = !down && N > 64;
+        const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
+        const uint32_t colG = 128u * s0;
+        const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+        if (!wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0)) break;
+        if (two && !wait_bar(acc_empty + s1, ((acc_ph >> s1) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s1)) break;
         ptx::tc_fence_after();
-        if (lane == 0) {
+        const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
+        const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
+        // the token scale atom covers the whole 128-row tile (row m in TMEM
+        // column m / 32); a chunk starting at row_off reads from column row_off / 32
+        const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
+        bool ok = true;
+        for (int st_i = 0; st_i < nsteps; ++st_i) {
+          if (!wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage)) { ok = false; break; }
+          ptx::tc_fence_after();
           uint8_t* st = smem + stage * S::kStride;
+          const int kb0 = st_i * j.nslab;
           if constexpr (kFp8) {
-            // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
-            ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
-            ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
-            if (!down || j.nslab == 2)
-              ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
-            if (down && j.nslab == 2)
-              ptx::tmem_cp_32x128b_x4(tmem + kColSfb1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb1), 16, 128, ptx::kLayoutNone));
+            if ((kb0 & 3) == 0) {   // a new group of four K blocks: its scale atoms
+              // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
+              ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
+              ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
+              if (!down)
+                ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
+            }
           }
           const uint64_t a0 = ptx::desc_kmajor_sw128(st);
           const uint64_t a1 = ptx::desc_kmajor_sw128(st + S::kOffA1);
           const uint64_t b0 = ptx::desc_kmajor_sw128(st + S::kOffB);
-          // the token scale atom covers the whole 128-row tile (row m in TMEM
-          // column m / 32); a chunk starting at row_off reads from column row_off / 32
-          const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
+          // scale-factor byte of a K block inside its atom: in the instruction
+          // descriptor and in the top two bits of the scale addresses
+          auto sfid = [](int kb) -> uint32_t { return (uint32_t)(kb & 3); };
           if (!down) {
+            const uint32_t id = sfid(kb0);
+            const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
+            const uint32_t sa0 = (tmem + kColSfa0) | (id << 30), sa1 = (tmem + kColSfa1) | (id << 30);
+            const uint32_t sb = (tmem + kColSfb0 + sfb_off) | (id << 30);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t acc = (st_i > 0 || kk > 0) ? 1u : 0u;
               const uint64_t off = (uint64_t)(kk * 32) >> 4;   // 32 bytes of K per MMA
               if constexpr (kFp8) {
-                ptx::mma_mxf8(tmem + colG, a0 + off, b0 + off, idesc, tmem + kColSfa0, tmem + kColSfb0 + sfb_off, acc);
-                ptx::mma_mxf8(tmem + colU, a1 + off, b0 + off, idesc, tmem + kColSfa1, tmem + kColSfb0 + sfb_off, acc);
+                ptx::mma_mxf8(tmem + colG, a0 + off, b0 + off, idesc_k, sa0, sb, acc);
+                ptx::mma_mxf8(tmem + colU, a1 + off, b0 + off, idesc_k, sa1, sb, acc);
               } else {
                 ptx::mma_f16(tmem + colG, a0 + off, b0 + off, idesc, acc);
                 ptx::mma_f16(tmem + colU, a1 + off, b0 + off, idesc, acc);
               }
             }
           } else {
-            for (int s = 0; s < j.nslab; ++s) {
-              const uint64_t as = s ? a1 : a0;
-              const uint64_t bs = ptx::desc_kmajor_sw128(st + S::kOffB + s * N * kSlab);
+            for (int sl = 0; sl < j.nslab; ++sl) {
+              const uint64_t as = sl ? a1 : a0;
+              const uint64_t bs = ptx::desc_kmajor_sw128(st + S::kOffB + sl * N * kSlab);
+              const uint32_t id = sfid(kb0 + sl);
+              const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
+              const uint32_t sa = (tmem + kColSfa0) | (id << 30);
+              const uint32_t sb = (tmem + kColSfb0 + sfb_off) | (id << 30);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (st_i > 0 || s > 0 || kk > 0) ? 1u : 0u;
+                const uint32_t acc = (st_i > 0 || sl > 0 || kk > 0) ? 1u : 0u;
                 const uint64_t off = (uint64_t)(kk * 32) >> 4;
                 if constexpr (kFp8) {
-                  ptx::mma_mxf8(tmem + colG, as + off, bs + off, idesc, tmem + (s ? kColSfa1 : kColSfa0),
-                                tmem + (s ? kColSfb1 : kColSfb0) + sfb_off, acc);
+                  ptx::mma_mxf8(tmem + colG, as + off, bs + off, idesc_k, sa, sb, acc);
                 } else {
                   ptx::mma_f16(tmem + colG, as + off, bs + off, idesc, acc);
                 }
@@ -560,22 +569,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             }
           }
           ptx::mma_commit(empty + stage);   // frees the stage once these MMAs are done
+          if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) break;
-      if (lane == 0) {
+        if (!ok) break;
         ptx::mma_commit(acc_full + s0);
         if (two) ptx::mma_commit(acc_full + s1);
+        acc_ph ^= 1u << s0;
+        if (two) acc_ph ^= 1u << s1;
+        else next_slot ^= 1u;
       }
-      __syncwarp();
-      acc_ph ^= 1u << s0;
-      if (two) acc_ph ^= 1u << s1;
-      else next_slot ^= 1u;
-    }
-    // drain: all MMAs and copies issued by this warp are complete
-    if (lane == 0) {
+      // drain: all MMAs and copies issued by this thread are complete
       ptx::mma_commit(drain);
       const unsigned long long t0 = globaltimer();
       while (!ptx::mbar_try_wait(drain, 0)) {
@@ -662,9 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             const int pe = pow2_scale_exp(amax);
             const int64_t r = row0 + n0 + f;
             p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
-            // scale atom of this tile and slice (row j.row_off + n0 + f of the tile)
-            *reinterpret_cast<uint32_t*>(p.ws.hsf + (tile_g * (p.I / 128) + j.slice) * kSfAtomBytes +
-                                         sf_atom_offset(j.row_off + n0 + f)) = (uint32_t)(pe + 127) * 0x01010101u;
+            // byte of this slice in the tile's scale atom (row j.row_off + n0 + f)
+            *sf_atom_byte(p.ws.hsf, tile_g, p.igroups, j.slice, j.row_off + n0 + f) = (uint8_t)(pe + 127);
           }
           ptx::named_barrier(1, 128);     // red[] is reused by the next batch
         } else {
@@ -779,6 +781,8 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.kelems = kel;
   p.nk1 = (int)(H / kel);
   p.nk2 = (int)(I / kel);
+  p.hgroups = (int)c.L.hgroups;
+  p.igroups = (int)c.L.igroups;
   p.tiles = c.L.tiles;
   ffn_tc_kernel<kFp8, kBRows><<<c.num_sms, kThreads, S::kSmemBytes, c.stream>>>(p);
   return cudaGetLastError();

@@ -31,9 +31,9 @@ constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
 // sentinel[E*tpe] u32 : (epoch << 8) | rows of a published tile
 // ring[E*tpe] u64     : (epoch << 32) | (e << 16) | tile, in publication order
 // xsf / hsf           : UE8M0 scale atoms of xq / hq for the block-scaled MMA,
-//                       [tile][128-value block][512 B]; row m of the tile owns
-//                       the 32-bit word at (m % 32) * 16 + (m / 32) * 4, all
-//                       four bytes holding the block's exponent
+//                       [tile][group of four 128-value blocks][512 B]; row m of
+//                       the tile owns the 32-bit word at (m % 32) * 16 +
+//                       (m / 32) * 4, byte b holding block 4 * group + b
 struct Header {
   uint32_t epoch_next;
   uint32_t epoch_cur;
@@ -47,7 +47,7 @@ enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kMiscWords = 8 };
 
 struct Layout {
   int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles = E * tpe
-  int64_t hblocks, iblocks;                 // H/128, I/128 (scale atoms per tile)
+  int64_t hgroups, igroups;                 // ceil(H/512), ceil(I/512): scale atoms per tile
   size_t set_words;                         // u32 words of one counter set
   size_t off_set[2], off_sentinel, off_ring, off_xsf, off_hsf, total;
 };
@@ -67,8 +67,8 @@ inline Layout make_layout(const moe_shape& s) {
   L.cap = default_cap(s);
   L.tpe = ceil_div(L.cap, kTileRows);
   L.tiles = L.E * L.tpe;
-  L.hblocks = ceil_div(L.H, kQBlock);
-  L.iblocks = ceil_div(L.I, kQBlock);
+  L.hgroups = ceil_div(L.H, 4 * kQBlock);
+  L.igroups = ceil_div(L.I, 4 * kQBlock);
   L.set_words = (size_t)(kMiscWords + L.E + 2 * L.tiles);
   size_t off = sizeof(Header);
   for (int i = 0; i < 2; ++i) {
@@ -80,10 +80,10 @@ inline Layout make_layout(const moe_shape& s) {
   L.off_ring = off;
   off = align_up(off + (size_t)L.tiles * 8, 256);
   L.off_xsf = off;
-  if (s.xq_dtype == MOE_E4M3) off = align_up(off + (size_t)L.tiles * L.hblocks * kSfAtomBytes, 256);
+  if (s.xq_dtype == MOE_E4M3) off = align_up(off + (size_t)L.tiles * L.hgroups * kSfAtomBytes, 256);
   L.off_hsf = off;
   if (s.h_dtype == MOE_E4M3 && !s.identity_experts)
-    off = align_up(off + (size_t)L.tiles * L.iblocks * kSfAtomBytes, 256);
+    off = align_up(off + (size_t)L.tiles * L.igroups * kSfAtomBytes, 256);
   L.total = off;
   return L;
 }
@@ -173,9 +173,16 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
 }
 
 // Byte offset of row m's 32-bit word inside one scale-factor atom of a
-// 128-row tile: 32 lanes x 16 bytes, lane m % 32, word m / 32.
+// 128-row tile: 32 lanes x 16 bytes, lane m % 32, word m / 32. Byte b of the
+// word holds block b of the atom's group of four.
 __device__ __forceinline__ int sf_atom_offset(int m) {
   return (m & 31) * 16 + (m >> 5) * 4;
+}
+
+// Scale atom (of xsf / hsf) of tile `tile` for 128-value block `blk`, and the
+// byte of row m in it.
+__device__ __forceinline__ uint8_t* sf_atom_byte(uint8_t* base, int64_t tile, int64_t groups, int blk, int m) {
+  return base + (tile * groups + blk / 4) * kSfAtomBytes + sf_atom_offset(m) + (blk & 3);
 }
 
 // Counter-set views.
