@@ -350,7 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         ptx::prefetch_tmap(&p.tm_h[b]);
       }
     }
-    const uint64_t pol = ptx::policy_evict_first();
+    // Weights: evict-first when each weight is read once (small tiles, one tile
+    // per expert); the normal policy when an expert's 2+ token tiles reuse the
+    // same weight slices through L2.
+    const uint64_t pol = kBRows <= 64 ? ptx::policy_evict_first() : ptx::policy_evict_normal();
     uint32_t stage = 0, phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per stage: a load is outstanding / its phase parity
     for (uint32_t i = 0;; ++i) {
