@@ -64,6 +64,23 @@ def dist_env():
         int(os.environ.get("WORLD_SIZE", 1))
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest of every rank's value (one all-reduce); the value itself
+    when there is no process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: the tokens of all ranks over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------ GPU clocks --
 
 class ClockSampler:
@@ -457,15 +474,9 @@ def run_ours(args):
     stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
                       for i in range(args.steps)])          # ms
     step_ms = stage.sum(1)
-    my_ms = float(step_ms.mean())
-    if world > 1:
-        t = torch.tensor([my_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    else:
-        ms = my_ms
+    ms = max_over_ranks(float(step_ms.mean()), dev)
     tokens_all = spec.T * world
-    value = tokens_all / (ms / 1000.0)
+    value = job_throughput(spec.T, world, ms)
 
     # end to end through the C ABI with host buffers: H2D of x and logits,
     # the layer, D2H of the output, every step
@@ -489,12 +500,8 @@ def run_ours(args):
             if i >= 2:
                 e_evs[i - 2][1].record(stream)
         torch.cuda.synchronize()
-        e_ms = statistics.mean(a.elapsed_time(z) for a, z in e_evs)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": tokens_all / (e_ms / 1000.0), "unit": "tokens/s",
+        e_ms = max_over_ranks(statistics.mean(a.elapsed_time(z) for a, z in e_evs), dev)
+        e2e = {"value": job_throughput(spec.T, world, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": hx.numel() * hx.element_size() + hl.numel() * hl.element_size(),
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
 

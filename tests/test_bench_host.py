@@ -1,0 +1,77 @@
+"""Host-side checks of bench.py that need no GPU: the multi-rank timing
+aggregation over a two-rank gloo group, and the reference arm (the CPU
+oracle) printing its JSON line."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = [2.0, 3.5][rank]                       # ms per step on this rank
+        ms = bench.max_over_ranks(mine)
+        out[rank] = (ms, bench.job_throughput(128, world, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    for rank in (0, 1):
+        ms, tput = res[rank]
+        assert ms == 3.5                              # the slowest rank's time
+        assert tput == pytest.approx(2 * 128 / 3.5e-3)   # all ranks' tokens
+
+
+def test_single_process_aggregation():
+    assert bench.max_over_ranks(1.25) == 1.25
+    assert bench.job_throughput(128, 1, 2.0) == pytest.approx(64000.0)
+
+
+def _run_bench(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True,
+                          text=True, timeout=300, env=env, cwd=ROOT)
+
+
+def test_reference_arm_prints_its_line():
+    r = _run_bench(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1",
+                    "--cpu-seconds", "0.5"])
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["higher_is_better"] is True
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                   {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
