@@ -9,8 +9,9 @@
 // Handshake"). Only counts, offsets and sync metadata are kept (Ascend report,
 // abstract).
 //
-// One CTA per token:
-//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j;
+// CTAs walk tokens; for each token:
+//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j (issued
+//     while the previous token's rows are being written);
 //  2. all warps stream the token row once (16-byte loads) and write it to the
 //     k claimed rows; E4M3 rows are quantised per 128 values with the
 //     smallest power-of-two scale that keeps the block within +-448, and the
@@ -18,7 +19,7 @@
 //     the block-scaled MMA;
 //  3. each slot bumps its tile's fill counter; the bump that completes 128 rows
 //     publishes the tile (sentinel + ring entry);
-//  4. the CTA that finishes the last token closes: it publishes the partial
+//  4. the last CTA to finish closes: it publishes the partial
 //     last tile of each expert, writes counts/offsets and the tile total, and
 //     advances the epoch.
 // Every CTA first zeroes its share of the counter set the *next* dispatch will
@@ -70,9 +71,106 @@ __device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e
                ((unsigned long long)epoch << 32) | ((unsigned long long)e << 16) | (unsigned)tile);
 }
 
+// Claim rows for the k slots of token t (threads tid < k); rows land in
+// s_row / s_e.
+__device__ __forceinline__ void claim_rows(const Args& a, int t, int tid, uint32_t* count, int* s_row,
+                                           int* s_e) {
+  if (tid >= a.k) return;
+  const int pair = t * a.k + tid;
+  const int e = __ldg(a.idx + pair);
+  int row = -1;
+  if (e >= 0 && e < a.E) {
+    const uint32_t p = atomicAdd(count + e, 1u);
+    if (p < (uint32_t)a.cap) {
+      row = e * a.cap + (int)p;
+      a.b.row_src[row] = pair;
+    } else {
+      latch_error(a.ws.hdr, MOE_ERR_CAPACITY, (uint32_t)e);
+    }
+  } else {
+    latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, (uint32_t)pair);
+  }
+  a.b.pos[pair] = row;
+  s_row[tid] = row;
+  s_e[tid] = e;
+}
+
+// Write token t's row to its claimed rows (all threads; a lane group of 8
+// covers one 128-value block). v0 holds this thread's first slice.
+__device__ __forceinline__ void stream_row(const Args& a, int t, int tid, const int* s_row, const float* v0) {
+  const int steps = a.H / kElems;
+  for (int s = tid; s < (steps + 31) / 32 * 32; s += kThreads) {
+    const bool live = s < steps;
+    const int h0 = s * kElems;
+    float v[kElems];
+    if (live && s == tid) {
+#pragma unroll
+      for (int i = 0; i < kElems; ++i) v[i] = v0[i];
+    } else if (live) {
+      load16(a.x, a.act, (int64_t)t * a.H + h0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kElems; ++i) v[i] = 0.f;
+    }
+    if (a.xq_dtype == MOE_E4M3) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < kElems; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      if (!live) continue;
+      const int p = pow2_scale_exp(amax);
+      const float inv = exp2i(-p > -126 ? -p : -126);  // 2^-p; p <= 120 for finite x
+      uint32_t q[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint16_t lo = cvt_e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv);
+        uint16_t hi = cvt_e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+        q[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+      }
+      const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+      const bool leader = (tid & 7) == 0;
+      const int blk = h0 / kQBlock;
+      for (int j = 0; j < a.k; ++j) {
+        const int row = s_row[j];
+        if (row < 0) continue;
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
+        if (leader) {
+          a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
+          if (a.xsf)   // tile id e * tpe + local = row / 128 since cap % 128 == 0
+            *sf_atom_byte(a.xsf, row / kTileRows, (a.H + 4 * kQBlock - 1) / (4 * kQBlock), blk,
+                          row % kTileRows) = (uint8_t)(p + 127);
+        }
+      }
+    } else if (live) {
+      for (int j = 0; j < a.k; ++j) {
+        const int row = s_row[j];
+        if (row < 0) continue;
+        const int64_t off = (int64_t)row * a.H + h0;
+        if (a.xq_dtype == MOE_BF16) {
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.b.xq) + off);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.b.xq) + off);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
-  __shared__ int s_row[kMaxTopk];
-  __shared__ int s_e[kMaxTopk];
+  __shared__ int s_row[2][kMaxTopk];   // double-buffered: this token's rows, the next token's
+  __shared__ int s_e[2][kMaxTopk];
   __shared__ uint32_t s_epoch;
   __shared__ int s_last;
   __shared__ uint32_t s_tiles;
@@ -94,123 +192,48 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     for (int64_t i = lo + tid; i < hi; i += kThreads) next[i] = 0u;
   }
 
-  const int t = blockIdx.x;
+  // Tokens blockIdx.x, + gridDim.x, ...: the next token's first row slice and
+  // row claims are issued before this token's rows are written, so their
+  // round trips overlap the streaming.
+  const int steps = a.H / kElems;
+  int cur = 0;
+  int t = blockIdx.x;
+  float v0[kElems];
   if (t < a.T) {
-    // the first slice of the row is read before the claims so the load and
-    // the atomics' round trips overlap
-    const int steps = a.H / kElems;
-    float v0[kElems];
     if (tid < steps) load16(a.x, a.act, (int64_t)t * a.H + tid * kElems, v0);
-
-    // 1. claim rows
-    if (tid < a.k) {
-      const int pair = t * a.k + tid;
-      const int e = __ldg(a.idx + pair);
-      int row = -1;
-      if (e >= 0 && e < a.E) {
-        const uint32_t p = atomicAdd(count + e, 1u);
-        if (p < (uint32_t)a.cap) {
-          row = e * a.cap + (int)p;
-          a.b.row_src[row] = pair;
-        } else {
-          latch_error(a.ws.hdr, MOE_ERR_CAPACITY, (uint32_t)e);
-        }
-      } else {
-        latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, (uint32_t)pair);
-      }
-      a.b.pos[pair] = row;
-      s_row[tid] = row;
-      s_e[tid] = e;
+    claim_rows(a, t, tid, count, s_row[0], s_e[0]);
+  }
+  __syncthreads();
+  for (; t < a.T; t += gridDim.x) {
+    const int tn = t + gridDim.x;
+    float vn[kElems];
+    if (tn < a.T) {
+      if (tid < steps) load16(a.x, a.act, (int64_t)tn * a.H + tid * kElems, vn);
+      claim_rows(a, tn, tid, count, s_row[cur ^ 1], s_e[cur ^ 1]);
     }
-    __syncthreads();
-
-    // 2. stream the row: lane group of 8 covers one 128-value block
-    for (int s = tid; s < (steps + 31) / 32 * 32; s += kThreads) {
-      const bool live = s < steps;
-      const int h0 = s * kElems;
-      float v[kElems];
-      if (live && s == tid) {
-#pragma unroll
-        for (int i = 0; i < kElems; ++i) v[i] = v0[i];
-      } else if (live) {
-        load16(a.x, a.act, (int64_t)t * a.H + h0, v);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kElems; ++i) v[i] = 0.f;
-      }
-      if (a.xq_dtype == MOE_E4M3) {
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < kElems; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-        if (!live) continue;
-        const int p = pow2_scale_exp(amax);
-        const float inv = exp2i(-p > -126 ? -p : -126);  // 2^-p; p <= 120 for finite x
-        uint32_t q[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint16_t lo = cvt_e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv);
-          uint16_t hi = cvt_e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv);
-          q[i] = (uint32_t)lo | ((uint32_t)hi << 16);
-        }
-        const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
-        const bool leader = (tid & 7) == 0;
-        const int blk = h0 / kQBlock;
-        for (int j = 0; j < a.k; ++j) {
-          const int row = s_row[j];
-          if (row < 0) continue;
-          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
-          if (leader) {
-            a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
-            if (a.xsf)   // tile id e * tpe + local = row / 128 since cap % 128 == 0
-              *sf_atom_byte(a.xsf, row / kTileRows, (a.H + 4 * kQBlock - 1) / (4 * kQBlock), blk,
-                            row % kTileRows) = (uint8_t)(p + 127);
-          }
-        }
-      } else if (live) {
-        for (int j = 0; j < a.k; ++j) {
-          const int row = s_row[j];
-          if (row < 0) continue;
-          const int64_t off = (int64_t)row * a.H + h0;
-          if (a.xq_dtype == MOE_BF16) {
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-              w[i] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.b.xq) + off);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.b.xq) + off);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          }
-        }
-      }
-    }
+    stream_row(a, t, tid, s_row[cur], v0);
     __threadfence();
     __syncthreads();
-
-    // 3. count the filled rows; the bump that completes a tile publishes it
+    // count the filled rows; the bump that completes a tile publishes it
     if (tid < a.k) {
-      const int row = s_row[tid];
+      const int row = s_row[cur][tid];
       if (row >= 0) {
-        const int e = s_e[tid];
+        const int e = s_e[cur][tid];
         const int local = row - e * a.cap;
         const int tile = local / kTileRows;
         const uint32_t old = atomicAdd(fill + (int64_t)e * a.tpe + tile, 1u);
         if (old + 1 == (uint32_t)kTileRows) publish_tile(a, set, epoch, e, tile, kTileRows);
       }
     }
+#pragma unroll
+    for (int i = 0; i < kElems; ++i) v0[i] = vn[i];
+    cur ^= 1;
+    __syncthreads();   // the next token's claims are visible; this token's rows are free
   }
   __threadfence();
   __syncthreads();
 
-  // 4. the last CTA closes
+  // the last CTA closes
   if (tid == 0) s_last = atomicAdd(misc + kDone, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!s_last) return;
@@ -256,7 +279,15 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
   a.ws = c.ws;
   a.xsf = write_sf && c.s.xq_dtype == MOE_E4M3 ? c.ws.xsf : nullptr;
   a.set_words = (int64_t)c.L.set_words;
-  const int grid = a.T > 0 ? a.T : 1;
+  // one wave of resident CTAs, each walking several tokens (fewer CTAs also
+  // means fewer arrivals on the closing counter)
+  static int resident = 0;
+  if (resident == 0) {
+    int r = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, dispatch_kernel, kThreads, 0) != cudaSuccess || r < 1) r = 1;
+    resident = r;
+  }
+  const int grid = a.T > 0 ? std::min(a.T, c.num_sms * resident) : 1;
   dispatch_kernel<<<grid, kThreads, 0, c.stream>>>(a);
   return cudaGetLastError();
 }
