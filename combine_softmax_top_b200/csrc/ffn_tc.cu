@@ -16,13 +16,14 @@
 // All gate/up units come before all down units; a down unit waits until the
 // I/128 gate/up units of its tile have stored h (per-slot counter).
 //
-// Per CTA (224 threads): warp 6 schedules jobs; warp 0 streams K slabs of 128 bytes into a 4- or 5-stage
-// shared-memory ring with TMA (weights with an evict-first hint), and for
-// e4m3 builds the weights' UE8M0 scale atoms and bulk-copies the tokens';
-// warp 1 issues tcgen05.mma (kind::f16 for bf16, kind::mxf8f6f4.block_scale
-// for e4m3) into tensor memory; warps 2-5 read the fp32 accumulators back with
+// Per CTA (352 threads): warp 10 schedules jobs; warp 0 streams K slabs of
+// 128 bytes into a 4- or 5-stage shared-memory ring with TMA, and for e4m3
+// builds the weights' UE8M0 scale atoms and bulk-copies the tokens'; warp 1
+// issues tcgen05.mma (kind::f16 for bf16, kind::mxf8f6f4.block_scale for
+// e4m3) into tensor memory; warps 2-9 read the fp32 accumulators back with
 // tcgen05.ld, apply SwiGLU and the per-128 requantisation (or round y to
-// bf16) and store. Every wait is bounded: on expiry the kernel latches
+// bf16) and store. The producer and MMA warps run warp-uniform loops and one
+// elected lane issues each copy, MMA and commit. Every wait is bounded: on expiry the kernel latches
 // MOE_ERR_TIMEOUT, drains its copies and MMAs, frees tensor memory and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -35,12 +36,14 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 224;   // warps: 0 TMA, 1 MMA, 2-5 epilogue, 6 scheduler
+constexpr int kThreads = 352;   // warps: 0 TMA, 1 MMA, 2-9 epilogue (two sets of four), 10 scheduler
+constexpr int kEpiThreads = 256;
+constexpr int kSchedWarp = 10;
 constexpr int kUQ = 8;          // unit-queue depth
 constexpr int kSlab = 128;      // K bytes per slab (one 128-byte swizzle row)
 constexpr int kABytes = 128 * kSlab;   // 128 weight rows of one slab
 constexpr int kMaxDynSmem = 232448;    // 227 KB per CTA
-constexpr int kCtlBytes = 1024;        // barriers, job queue, flags, reductions
+constexpr int kCtlBytes = 2048;        // barriers, job queue, flags, reductions
 constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert first-tile table (E <= 1024)
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
@@ -198,7 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   int4* epi_job = reinterpret_cast<int4*>(ctl + 384);          // job broadcast to the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 400);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 404);
-  float* red = reinterpret_cast<float*>(ctl + 512);            // [4 warps][32 tokens]
+  float* red = reinterpret_cast<float*>(ctl + 512);            // [2 sets][4 warps][32 tokens]
+  float* sinv = reinterpret_cast<float*>(ctl + 1536);          // [2 sets][32 tokens] 1 / scale
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -248,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     return true;
   };
 
-  if (warp == 6) {
+  if (warp == kSchedWarp) {
     // ---------------------------------------------------------------- scheduler
     // Units, expert-major: for each expert, for each 128-feature slice, every
     // tile of that expert (all gate/up units before all down units), dealt
@@ -433,7 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           }
           __syncwarp();
         }
-        if (lane == 0) {
+        // one elected lane issues the copies; every operand is warp-uniform
+        if (ptx::elect_one()) {
           ptx::mbar_arrive_expect_tx(full + stage, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
           if (down) {
             for (int s = 0; s < j.nslab; ++s)
@@ -492,33 +497,50 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // Two 128-column accumulator slots: a job with N <= 64 (or a down job)
     // takes one (gate at +0, up at +64), a gate/up job with N > 64 takes both,
     // so the next job's MMAs overlap the previous job's epilogue.
-    // One thread issues everything (the other lanes wait at the end): no
-    // warp-wide shuffles or syncs per K step.
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0, acc_ph = 0 /* bit per slot */, next_slot = 0;
-      for (uint32_t i = 0;; ++i) {
-        Job j;
-        if (!take_job(i, &j) || j.kind >= kKindEnd) break;
-        const bool down = j.kind == kKindDown;
-        const int N = (j.rows + 15) & ~15;
-        const bool two = !down && N > 64;
-        const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
-        const uint32_t colG = 128u * s0;
-        const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
-        if (!wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0)) break;
-        if (two && !wait_bar(acc_empty + s1, ((acc_ph >> s1) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s1)) break;
+    // The whole warp walks the loop with warp-uniform values (descriptors,
+    // tensor-memory addresses); lane 0 polls the barriers and one elected
+    // lane issues the copies, MMAs and commits.
+    uint32_t stage = 0, phase = 0, acc_ph = 0 /* bit per slot */, next_slot = 0;
+    for (uint32_t i = 0;; ++i) {
+      int4 raw = make_int4(0, 0, kKindAbort << 16, 0);
+      if (lane == 0) {
+        Job jj;
+        if (take_job(i, &jj)) raw = pack_job(jj);
+      }
+      const Job j = unpack_job(shfl_int4(raw));
+      if (j.kind >= kKindEnd) break;
+      const bool down = j.kind == kKindDown;
+      const int N = (j.rows + 15) & ~15;
+      const bool two = !down && N > 64;
+      const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
+      const uint32_t colG = 128u * s0;
+      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+      int ok = 1;
+      if (lane == 0) {
+        ok = wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0);
+        if (ok && two) ok = wait_bar(acc_empty + s1, ((acc_ph >> s1) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s1);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      ptx::tc_fence_after();
+      const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
+      const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
+      // the token scale atom covers the whole 128-row tile (row m in TMEM
+      // column m / 32); a chunk starting at row_off reads from column row_off / 32
+      const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
+      for (int st_i = 0; st_i < nsteps; ++st_i) {
+        int w_ok = 1;
+        if (lane == 0) w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage);
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = 0; break; }
         ptx::tc_fence_after();
-        const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
-        const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
-        // the token scale atom covers the whole 128-row tile (row m in TMEM
-        // column m / 32); a chunk starting at row_off reads from column row_off / 32
-        const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
-        bool ok = true;
-        for (int st_i = 0; st_i < nsteps; ++st_i) {
-          if (!wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage)) { ok = false; break; }
-          ptx::tc_fence_after();
-          uint8_t* st = smem + stage * S::kStride;
-          const int kb0 = st_i * j.nslab;
+        uint8_t* st = smem + stage * S::kStride;
+        const int kb0 = st_i * j.nslab;
+        const uint64_t a0 = ptx::desc_kmajor_sw128(st);
+        const uint64_t a1 = ptx::desc_kmajor_sw128(st + S::kOffA1);
+        const uint64_t b0 = ptx::desc_kmajor_sw128(st + S::kOffB);
+        // scale-factor byte of a K block inside its atom: in the instruction
+        // descriptor and in the top two bits of the scale addresses
+        auto sfid = [](int kb) -> uint32_t { return (uint32_t)(kb & 3); };
+        if (ptx::elect_one()) {
           if constexpr (kFp8) {
             if ((kb0 & 3) == 0) {   // a new group of four K blocks: its scale atoms
               // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
@@ -528,12 +550,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
                 ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
             }
           }
-          const uint64_t a0 = ptx::desc_kmajor_sw128(st);
-          const uint64_t a1 = ptx::desc_kmajor_sw128(st + S::kOffA1);
-          const uint64_t b0 = ptx::desc_kmajor_sw128(st + S::kOffB);
-          // scale-factor byte of a K block inside its atom: in the instruction
-          // descriptor and in the top two bits of the scale addresses
-          auto sfid = [](int kb) -> uint32_t { return (uint32_t)(kb & 3); };
           if (!down) {
             const uint32_t id = sfid(kb0);
             const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
@@ -572,16 +588,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             }
           }
           ptx::mma_commit(empty + stage);   // frees the stage once these MMAs are done
-          if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        if (++stage == (uint32_t)kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (ptx::elect_one()) {
         ptx::mma_commit(acc_full + s0);
         if (two) ptx::mma_commit(acc_full + s1);
-        acc_ph ^= 1u << s0;
-        if (two) acc_ph ^= 1u << s1;
-        else next_slot ^= 1u;
       }
-      // drain: all MMAs and copies issued by this thread are complete
+      __syncwarp();
+      acc_ph ^= 1u << s0;
+      if (two) acc_ph ^= 1u << s1;
+      else next_slot ^= 1u;
+    }
+    // drain: all MMAs and copies issued by the elected lane are complete
+    if (ptx::elect_one()) {
       ptx::mma_commit(drain);
       const unsigned long long t0 = globaltimer();
       while (!ptx::mbar_try_wait(drain, 0)) {
@@ -591,9 +613,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
+    // Eight warps in two sets of four; warp w reads TMEM lanes 32 (w % 4) ..
+    // +31 (output features), and set s takes the 32-token batches s, s + 2, ..
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int f = q * 32 + lane;            // output feature within the slice
-    const int et = threadIdx.x - 64;        // 0..127
+    const int et = threadIdx.x - 64;        // 0..255
+    const int set = et >> 7;                // 0 or 1
+    const uint32_t set_bar = 2u + (uint32_t)set;   // named barrier of the set (128 threads)
+    float* red_s = red + set * 128;
+    float* sinv_s = sinv + set * 32;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t acc_ph = 0, next_slot = 0;
     for (uint32_t i = 0;; ++i) {
@@ -611,9 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         }
         *epi_job = pack_job(jj);
       }
-      ptx::named_barrier(1, 128);
+      ptx::named_barrier(1, kEpiThreads);
       const Job j = unpack_job(*epi_job);
-      ptx::named_barrier(1, 128);
+      ptx::named_barrier(1, kEpiThreads);
       if (j.kind >= kKindEnd) break;
       const bool down = j.kind == kKindDown;
       const int N = (j.rows + 15) & ~15;
@@ -628,8 +656,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
       // tokens in batches of 32 columns: one TMEM load per operand, the
       // per-token max over this warp's 32 features in one redux, the max over
-      // the four warps through shared memory
-      for (int n0 = 0; n0 < j.rows; n0 += 32) {
+      // the set's four warps and the scale once per token through shared memory
+      for (int n0 = 32 * set; n0 < j.rows; n0 += 64) {
         uint32_t g[32], uu[32];
         ptx::tmem_ld_x32(tmem + lane_base + colG + n0, g);
         if (!down) ptx::tmem_ld_x32(tmem + lane_base + colU + n0, uu);
@@ -650,28 +678,34 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[jj])));
-            if (lane == jj) red[q * 32 + jj] = __uint_as_float(m);
+            if (lane == jj) red_s[q * 32 + jj] = __uint_as_float(m);
           }
-          ptx::named_barrier(1, 128);
-          uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const float amax = fmaxf(fmaxf(red[jj], red[32 + jj]), fmaxf(red[64 + jj], red[96 + jj]));
+          ptx::named_barrier(set_bar, 128);
+          if (q == 0) {   // lane t: token n0 + t's scale over the 128 features
+            const float amax = fmaxf(fmaxf(red_s[lane], red_s[32 + lane]), fmaxf(red_s[64 + lane], red_s[96 + lane]));
             const int pe = pow2_scale_exp(amax);
-            if (jj < nv) {
-              const uint16_t b2 = cvt_e4m3x2(h[jj] * exp2i(-pe > -126 ? -pe : -126), 0.f);
-              hp[(int64_t)jj * p.I] = (uint8_t)(b2 & 0xFF);
+            sinv_s[lane] = exp2i(-pe > -126 ? -pe : -126);
+            if (lane < nv) {
+              const int64_t r = row0 + n0 + lane;
+              p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
+              // byte of this slice in the tile's scale atom (row j.row_off + n0 + lane)
+              *sf_atom_byte(p.ws.hsf, tile_g, p.igroups, j.slice, j.row_off + n0 + lane) = (uint8_t)(pe + 127);
             }
           }
-          if (f < nv) {   // thread f records token f's scale
-            const float amax = fmaxf(fmaxf(red[f], red[32 + f]), fmaxf(red[64 + f], red[96 + f]));
-            const int pe = pow2_scale_exp(amax);
-            const int64_t r = row0 + n0 + f;
-            p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
-            // byte of this slice in the tile's scale atom (row j.row_off + n0 + f)
-            *sf_atom_byte(p.ws.hsf, tile_g, p.igroups, j.slice, j.row_off + n0 + f) = (uint8_t)(pe + 127);
+          ptx::named_barrier(set_bar, 128);
+          uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
+          const float4* sv = reinterpret_cast<const float4*>(sinv_s);
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 v = sv[j4];
+            const float inv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int jj = 4 * j4 + b;
+              if (jj < nv) hp[(int64_t)jj * p.I] = (uint8_t)(cvt_e4m3x2(h[jj] * inv[b], 0.f) & 0xFF);
+            }
           }
-          ptx::named_barrier(1, 128);     // red[] is reused by the next batch
+          ptx::named_barrier(set_bar, 128);     // red / sinv are reused by the next batch
         } else {
           __nv_bfloat16* hp = reinterpret_cast<__nv_bfloat16*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
@@ -681,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       }
       // accumulators consumed: let the MMA warp reuse the slot(s)
       ptx::tc_fence_before();
-      ptx::named_barrier(1, 128);
+      ptx::named_barrier(1, kEpiThreads);
       if (et == 0) {
         ptx::mbar_arrive(acc_empty + s0);
         if (two) ptx::mbar_arrive(acc_empty + s1);
@@ -692,12 +726,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       if (!down) {
         // publish this chunk of this slice of h to the down jobs of the tile
         __threadfence();
-        ptx::named_barrier(1, 128);
+        ptx::named_barrier(1, kEpiThreads);
         if (et == 0) atomicAdd(hdone + j.slot, 1u);
       }
     }
   }
-
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
