@@ -355,9 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       }
     }
     // Weights: evict-first when each weight is read once (small tiles, one tile
-    // per expert); the normal policy when an expert's 2+ token tiles reuse the
+    // per expert); the default policy when an expert's 2+ token tiles reuse the
     // same weight slices through L2.
-    const uint64_t pol = kBRows <= 64 ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+    const uint64_t pol = ptx::policy_evict_first();
     uint32_t stage = 0, phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per stage: a load is outstanding / its phase parity
     for (uint32_t i = 0;; ++i) {
@@ -405,7 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         return w;
       };
       if constexpr (kFp8) load_scales(0);
-      const CUtensorMap* tmb = down ? p.tm_h : p.tm_x;   // 16-row boxes
       bool ok = true;
       for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
@@ -437,41 +436,58 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           }
           __syncwarp();
         }
-        // one elected lane issues the copies; every operand is warp-uniform
+        // one elected lane issues the copies; every operand is warp-uniform.
+        // Each copy names its tensor map at a fixed parameter address: a map
+        // chosen at run time costs about four times as much to issue.
         if (ptx::elect_one()) {
-          ptx::mbar_arrive_expect_tx(full + stage, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
+          uint64_t* fb = full + stage;
+          ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
+          const int kx0 = kb0 * p.kelems;
           if (down) {
-            for (int s = 0; s < j.nslab; ++s)
-              ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, full + stage, (kb0 + s) * p.kelems, arow, pol);
-          } else {
-            ptx::tma_load_2d_hint(st, &p.tm_wg, full + stage, kb0 * p.kelems, arow, pol);
-            ptx::tma_load_2d_hint(st + S::kOffA1, &p.tm_wu, full + stage, kb0 * p.kelems, arow, pol);
+            for (int s = 0; s < j.nslab; ++s) {
+              if constexpr (kBRows <= 64)
+                ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow, pol);
+              else
+                ptx::tma_load_2d(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow);
+            }
+          } else if constexpr (kBRows <= 64) {
+            ptx::tma_load_2d_hint(st, &p.tm_wg, fb, kx0, arow, pol);
+            ptx::tma_load_2d_hint(st + S::kOffA1, &p.tm_wu, fb, kx0, arow, pol);
+          } else {   // default policy: an expert's token tiles reuse the slice through L2
+            ptx::tma_load_2d(st, &p.tm_wg, fb, kx0, arow);
+            ptx::tma_load_2d(st + S::kOffA1, &p.tm_wu, fb, kx0, arow);
           }
-          // token rows in the largest boxes that fit: N = 128/64/32/16-row pieces
-          // Small tiles (decode) go in 16-row boxes, large ones in the fewest
-          // boxes of 128/64/32/16 rows; measured, each is the faster choice
-          // for its variant.
-          if constexpr (kBRows <= 64) {
-            for (int s = 0; s < j.nslab; ++s)
-              for (int r = 0; r < N / 16; ++r)
-                ptx::tma_load_2d(st + S::kOffB + s * N * kSlab + r * 2048, tmb, full + stage, (kb0 + s) * p.kelems,
-                                 brow + 16 * r);
-          }
-          for (int s = 0; kBRows > 64 && s < j.nslab; ++s) {
+          // token rows: small tiles (decode) in 16-row boxes, large ones in
+          // the fewest boxes of 128/64/32/16 rows; measured, each is the
+          // faster choice for its variant
+          for (int s = 0; s < j.nslab; ++s) {
             uint8_t* dst = st + S::kOffB + s * N * kSlab;
-            const int kx = (kb0 + s) * p.kelems;
-            {
+            const int kx = kx0 + s * p.kelems;
+            if constexpr (kBRows <= 64) {
+              if (down) {
+                for (int r = 0; r < N / 16; ++r) ptx::tma_load_2d(dst + r * 2048, &p.tm_h[0], fb, kx, brow + 16 * r);
+              } else {
+                for (int r = 0; r < N / 16; ++r) ptx::tma_load_2d(dst + r * 2048, &p.tm_x[0], fb, kx, brow + 16 * r);
+              }
+            } else if (N == 128) {   // the common full tile: one box
+              if (down) ptx::tma_load_2d(dst, &p.tm_h[3], fb, kx, brow);
+              else ptx::tma_load_2d(dst, &p.tm_x[3], fb, kx, brow);
+            } else if (down) {
               int r = 0;
-              if (N - r >= 128) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[3] : &p.tm_x[3], full + stage, kx, brow + r); r += 128; }
-              if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[2] : &p.tm_x[2], full + stage, kx, brow + r); r += 64; }
-              if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[1] : &p.tm_x[1], full + stage, kx, brow + r); r += 32; }
-              if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, down ? &p.tm_h[0] : &p.tm_x[0], full + stage, kx, brow + r); r += 16; }
+              if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[2], fb, kx, brow + r); r += 64; }
+              if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[1], fb, kx, brow + r); r += 32; }
+              if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[0], fb, kx, brow + r); r += 16; }
+            } else {
+              int r = 0;
+              if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[2], fb, kx, brow + r); r += 64; }
+              if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[1], fb, kx, brow + r); r += 32; }
+              if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[0], fb, kx, brow + r); r += 16; }
             }
           }
           if (sf_stage) {   // the tokens' scale atom of this group of four blocks
             const uint8_t* sf = down ? p.ws.hsf + (tile_g * p.igroups + kb0 / 4) * kSfAtomBytes
                                      : p.ws.xsf + (tile_g * p.hgroups + kb0 / 4) * kSfAtomBytes;
-            ptx::bulk_load(st + S::kOffSfb0, sf, kSfAtomBytes, full + stage);
+            ptx::bulk_load(st + S::kOffSfb0, sf, kSfAtomBytes, fb);
           }
         }
         __syncwarp();
