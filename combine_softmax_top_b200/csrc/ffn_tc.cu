@@ -12,7 +12,8 @@
 //
 // Work units, processed in one fixed order by a persistent grid:
 //   gate/up : (ring slot, 128-feature slice of I) -> h rows of that slice
-//   down    : (ring slot, 128-feature slice of H) -> y rows of that slice
+//   down    : (ring slot, 128-feature slice of H, or two slices sharing the
+//             token tile when tiles hold up to 128 rows) -> y rows
 // All gate/up units come before all down units; a down unit waits until the
 // I/128 gate/up units of its tile have stored h (per-slot counter).
 //
@@ -91,11 +92,12 @@ struct TcParams {
 // slice, in one phase.
 struct Job {
   int e, tile, slice, rows, row_off, kind, nslab, slot;
+  int pair;   // down job over two 128-feature slices of H (slice, slice + 1)
 };
 
 __device__ __forceinline__ int4 pack_job(const Job& j) {
   return make_int4(j.e, j.tile | (j.slice << 16),
-                   j.rows | (j.row_off << 8) | (j.kind << 16) | (j.nslab << 20), j.slot);
+                   j.rows | (j.row_off << 8) | (j.kind << 16) | (j.nslab << 20) | (j.pair << 24), j.slot);
 }
 
 __device__ __forceinline__ Job unpack_job(int4 v) {
@@ -107,6 +109,7 @@ __device__ __forceinline__ Job unpack_job(int4 v) {
   j.row_off = (v.z >> 8) & 0xFF;
   j.kind = (v.z >> 16) & 0xF;
   j.nslab = (v.z >> 20) & 0xF;
+  j.pair = (v.z >> 24) & 0x1;
   j.slot = v.w;
   return j;
 }
@@ -239,8 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   const uint32_t ntiles = ld_acquire(misc + kRingTotal);
   const uint32_t gen = ld_acquire(misc + kFfnGen);   // FFN calls already made on this dispatch
   uint32_t* hdone = set_hdone(set, p.E, p.tiles);
+  // down units cover two slices of H each when tiles are large (the two share
+  // the token tile, like gate and up)
+  const int dpair = (kBRows > 64 && (p.n_hslices & 1) == 0) ? 2 : 1;
   const uint32_t n1 = ntiles * (uint32_t)p.n_islices;
-  const uint32_t total = n1 + ntiles * (uint32_t)p.n_hslices;
+  const uint32_t total = n1 + ntiles * (uint32_t)(p.n_hslices / dpair);
   Header* hdr = p.ws.hdr;
 
   // Take job i from the queue (one lane of a consumer role).
@@ -307,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         Job j;
         j.kind = u >= n1 ? kKindDown : kKindGateUp;
         const uint32_t v = j.kind == kKindDown ? u - n1 : u;
-        const uint32_t ns = (uint32_t)(j.kind == kKindDown ? p.n_hslices : p.n_islices);
+        const uint32_t ns = (uint32_t)(j.kind == kKindDown ? p.n_hslices / dpair : p.n_islices);
         // expert: the last e with tile_pre[e] * ns <= v (empty experts never are)
         int lo = 0, hi = p.E - 1;
         while (lo < hi) {
@@ -318,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         j.e = lo;
         const uint32_t nt = (uint32_t)(tile_pre[lo + 1] - tile_pre[lo]);
         const uint32_t w = v - (uint32_t)tile_pre[lo] * ns;
-        j.slice = (int)(w / nt);
+        j.pair = j.kind == kKindDown && dpair == 2;
+        j.slice = (int)(w / nt) * (j.pair ? 2 : 1);
         j.tile = (int)(w % nt);
         j.slot = j.e * p.tpe + j.tile;     // global tile id: the down units' counter
         int rows = 0;
@@ -332,12 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           j.row_off = c * kBRows;
           j.rows = min(kBRows, rows - j.row_off);
           const int N = (j.rows + 15) & ~15;
-          j.nslab = (j.kind == kKindDown && 2 * N <= kBRows && (p.nk2 & 1) == 0) ? 2 : 1;
+          j.nslab = (j.kind == kKindDown && !j.pair && 2 * N <= kBRows && (p.nk2 & 1) == 0) ? 2 : 1;
           good = push(j);
         }
       }
       Job end;
-      end.e = end.tile = end.slice = end.rows = end.row_off = end.slot = 0;
+      end.e = end.tile = end.slice = end.rows = end.row_off = end.slot = end.pair = 0;
       end.nslab = 1;
       end.kind = good ? kKindEnd : kKindAbort;
       push(end);   // bounded; consumers also stop on the abort flag
@@ -375,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int arow = j.e * (down ? p.H : p.I) + j.slice * 128;
       const int brow = j.e * p.cap + j.tile * kTileRows + j.row_off;
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
-      const uint32_t tx = (down ? (uint32_t)j.nslab : 2u) * kABytes + (uint32_t)(j.nslab * N * kSlab);
+      const bool dual = !down || j.pair;   // two weight tiles share the token tile
+      const uint32_t tx = (dual ? 2u : (uint32_t)j.nslab) * kABytes + (uint32_t)(j.nslab * N * kSlab);
       // the job's weight scales, one per 128 x 128 block along K: lane l holds
       // the exponents of blocks l and l + 32 (gate/down in sa, up in sb), read
       // once per job
@@ -384,11 +392,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int nkb = down ? p.I / 128 : p.H / 128;
       const float* pa = down ? p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * nkb
                              : p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
-      const float* pb = p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      const float* pb = down ? p.sd + ((int64_t)j.e * p.n_hslices + j.slice + 1) * nkb
+                             : p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
       auto load_scales = [&](int base) {
         if (lane + base < nkb) sa0 = ue8m0(__ldg(pa + base + lane));
         if (lane + base + 32 < nkb) sa1 = ue8m0(__ldg(pa + base + lane + 32));
-        if (!down) {
+        if (dual) {
           if (lane + base < nkb) sb0 = ue8m0(__ldg(pb + base + lane));
           if (lane + base + 32 < nkb) sb1 = ue8m0(__ldg(pb + base + lane + 32));
         }
@@ -428,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             const int kr = kb0 - sbase;
             const uint32_t w0 = pack4(sa0, sa1, kr);
             reinterpret_cast<uint4*>(st + S::kOffSfa0)[lane] = make_uint4(w0, w0, w0, w0);
-            if (!down) {
+            if (dual) {
               const uint32_t w1 = pack4(sb0, sb1, kr);
               reinterpret_cast<uint4*>(st + S::kOffSfa1)[lane] = make_uint4(w1, w1, w1, w1);
             }
@@ -444,11 +453,17 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
           const int kx0 = kb0 * p.kelems;
           if (down) {
-            for (int s = 0; s < j.nslab; ++s) {
-              if constexpr (kBRows <= 64)
+            if constexpr (kBRows <= 64) {
+              for (int s = 0; s < j.nslab; ++s)
                 ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow, pol);
-              else
-                ptx::tma_load_2d(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow);
+            } else {   // one slab of slices (slice, slice + 1), or nslab slabs of one slice
+              if (j.pair) {
+                ptx::tma_load_2d(st, &p.tm_wd, fb, kx0, arow);
+                ptx::tma_load_2d(st + S::kOffA1, &p.tm_wd, fb, kx0, arow + 128);
+              } else {
+                for (int s = 0; s < j.nslab; ++s)
+                  ptx::tma_load_2d(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow);
+              }
             }
           } else if constexpr (kBRows <= 64) {
             ptx::tma_load_2d_hint(st, &p.tm_wg, fb, kx0, arow, pol);
@@ -526,8 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const Job j = unpack_job(shfl_int4(raw));
       if (j.kind >= kKindEnd) break;
       const bool down = j.kind == kKindDown;
+      const bool dual = !down || j.pair;   // two accumulators: gate/up or two slices of H
       const int N = (j.rows + 15) & ~15;
-      const bool two = !down && N > 64;
+      const bool two = dual && N > 64;
       const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
       const uint32_t colG = 128u * s0;
       const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
@@ -562,11 +578,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
               ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
               ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
-              if (!down)
+              if (dual)
                 ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
             }
           }
-          if (!down) {
+          if (dual) {
             const uint32_t id = sfid(kb0);
             const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
             const uint32_t sa0 = (tmem + kColSfa0) | (id << 30), sa1 = (tmem + kColSfa1) | (id << 30);
@@ -647,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         if (!good) jj.kind = kKindAbort;
         if (jj.kind < kKindEnd) {
           const int N = (jj.rows + 15) & ~15;
-          const bool two = jj.kind == kKindGateUp && N > 64;
+          const bool two = (jj.kind == kKindGateUp || jj.pair) && N > 64;
           const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
           good = wait_bar(acc_full + s0, (acc_ph >> s0) & 1u, abort_flag, hdr, 0x70000000u | s0);
           if (good && two) good = wait_bar(acc_full + s1, (acc_ph >> s1) & 1u, abort_flag, hdr, 0x70000000u | s1);
@@ -660,8 +676,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ptx::named_barrier(1, kEpiThreads);
       if (j.kind >= kKindEnd) break;
       const bool down = j.kind == kKindDown;
+      const bool dual = !down || j.pair;
       const int N = (j.rows + 15) & ~15;
-      const bool two = !down && N > 64;
+      const bool two = dual && N > 64;
       const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
       const uint32_t colG = 128u * s0;
       const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
@@ -670,30 +687,68 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ptx::tc_fence_after();
       const int64_t row0 = (int64_t)j.e * p.cap + (int64_t)j.tile * kTileRows + j.row_off;
       const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
-      // tokens in batches of 32 columns: one TMEM load per operand, the
-      // per-token max over this warp's 32 features in one redux, the max over
-      // the set's four warps and the scale once per token through shared memory
-      for (int n0 = 32 * set; n0 < j.rows; n0 += 64) {
-        uint32_t g[32], uu[32];
-        ptx::tmem_ld_x32(tmem + lane_base + colG + n0, g);
-        if (!down) ptx::tmem_ld_x32(tmem + lane_base + colU + n0, uu);
-        ptx::tmem_wait_ld();
-        const int nv = min(32, j.rows - n0);
+      // Set s owns the 32-token batches at columns 32 s and 32 s + 64 (a job
+      // has at most 128 rows). Both are drained from TMEM into registers first
+      // -- h = SwiGLU in fp32, or y already rounded to bf16 (two slices packed
+      // per word) -- and the accumulators are released before any of the
+      // slower per-token work, so the next job's MMAs overlap all of it.
+      const int nA = max(0, min(32, j.rows - 32 * set));
+      const int nB = max(0, min(32, j.rows - 32 * set - 64));
+      uint32_t vA[32], vB[32];
+      auto drain = [&](int n0, uint32_t (&v)[32]) {
+#pragma unroll
+        for (int hh = 0; hh < 32; hh += 16) {   // 16 columns at a time: fewer live registers
+          uint32_t g[16], uu[16];
+          ptx::tmem_ld_x16(tmem + lane_base + colG + n0 + hh, g);
+          if (dual) ptx::tmem_ld_x16(tmem + lane_base + colU + n0 + hh, uu);
+          ptx::tmem_wait_ld();
+          if (down) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(g[jj]), dual ? __uint_as_float(uu[jj]) : 0.f);
+              v[hh + jj] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              v[hh + jj] = __float_as_uint(silu(__uint_as_float(g[jj])) * __uint_as_float(uu[jj]));
+          }
+        }
+      };
+      if (nA > 0) drain(32 * set, vA);
+      if (nB > 0) drain(32 * set + 64, vB);
+      // accumulators consumed: let the MMA warp reuse the slot(s)
+      ptx::tc_fence_before();
+      ptx::named_barrier(1, kEpiThreads);
+      if (et == 0) {
+        ptx::mbar_arrive(acc_empty + s0);
+        if (two) ptx::mbar_arrive(acc_empty + s1);
+      }
+      acc_ph ^= 1u << s0;
+      if (two) acc_ph ^= 1u << s1;
+      else next_slot ^= 1u;
+      // the per-token work on one drained batch: y stores, or the per-token
+      // max over the 128 features (one redux per token per warp, the max over
+      // the set's four warps and the scale once per token through shared
+      // memory), requantisation and h stores
+      auto finish = [&](int n0, int nv, const uint32_t (&v)[32]) {
         if (down) {
           __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(p.y) + (row0 + n0) * p.H + j.slice * 128 + f;
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj)
-            if (jj < nv) yp[(int64_t)jj * p.H] = __float2bfloat16_rn(__uint_as_float(g[jj]));
-          continue;
-        }
-        float h[32];
+            if (jj < nv) yp[(int64_t)jj * p.H] = __ushort_as_bfloat16((unsigned short)(v[jj] & 0xFFFFu));
+          if (j.pair) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) h[jj] = silu(__uint_as_float(g[jj])) * __uint_as_float(uu[jj]);
+            for (int jj = 0; jj < 32; ++jj)
+              if (jj < nv) yp[(int64_t)jj * p.H + 128] = __ushort_as_bfloat16((unsigned short)(v[jj] >> 16));
+          }
+          return;
+        }
         if constexpr (kFp8) {
           // |h| bit patterns order like the values (non-negative floats)
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
-            const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[jj])));
+            const uint32_t m = __reduce_max_sync(0xffffffffu, v[jj] & 0x7FFFFFFFu);
             if (lane == jj) red_s[q * 32 + jj] = __uint_as_float(m);
           }
           ptx::named_barrier(set_bar, 128);
@@ -713,12 +768,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           const float4* sv = reinterpret_cast<const float4*>(sinv_s);
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 v = sv[j4];
-            const float inv[4] = {v.x, v.y, v.z, v.w};
+            const float4 iv = sv[j4];
+            const float inv[4] = {iv.x, iv.y, iv.z, iv.w};
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const int jj = 4 * j4 + b;
-              if (jj < nv) hp[(int64_t)jj * p.I] = (uint8_t)(cvt_e4m3x2(h[jj] * inv[b], 0.f) & 0xFF);
+              if (jj < nv) hp[(int64_t)jj * p.I] = (uint8_t)(cvt_e4m3x2(__uint_as_float(v[jj]) * inv[b], 0.f) & 0xFF);
             }
           }
           ptx::named_barrier(set_bar, 128);     // red / sinv are reused by the next batch
@@ -726,19 +781,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           __nv_bfloat16* hp = reinterpret_cast<__nv_bfloat16*>(p.hq) + (row0 + n0) * p.I + j.slice * 128 + f;
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj)
-            if (jj < nv) hp[(int64_t)jj * p.I] = __float2bfloat16_rn(h[jj]);
+            if (jj < nv) hp[(int64_t)jj * p.I] = __float2bfloat16_rn(__uint_as_float(v[jj]));
         }
-      }
-      // accumulators consumed: let the MMA warp reuse the slot(s)
-      ptx::tc_fence_before();
-      ptx::named_barrier(1, kEpiThreads);
-      if (et == 0) {
-        ptx::mbar_arrive(acc_empty + s0);
-        if (two) ptx::mbar_arrive(acc_empty + s1);
-      }
-      acc_ph ^= 1u << s0;
-      if (two) acc_ph ^= 1u << s1;
-      else next_slot ^= 1u;
+      };
+      if (nA > 0) finish(32 * set, nA, vA);
+      if (nB > 0) finish(32 * set + 64, nB, vB);
       if (!down) {
         // publish this chunk of this slice of h to the down jobs of the tile
         __threadfence();
