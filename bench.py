@@ -158,14 +158,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle --
 
-def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None):
+def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None, threads: int | None = None):
     """Time the CPU oracle on the first tokens of the workload until `seconds`
-    of wall time are spent. Returns (tokens, elapsed_s, cores)."""
+    of wall time are spent, on all host cores or on `threads` of them.
+    Returns (tokens, elapsed_s, cores)."""
     import numpy as np
     import torch
     import oracle
 
-    cores = len(os.sched_getaffinity(0))
+    all_cores = len(os.sched_getaffinity(0))
+    cores = oracle.set_threads(threads if threads else all_cores)
     odt = {"f32": oracle.F32, "bf16": oracle.BF16, "e4m3": oracle.E4M3}
 
     def host(t):
@@ -195,6 +197,7 @@ def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None):
         oracle.moe_layer(p, x, logits, done, t1)
         elapsed += time.perf_counter() - t_start
         done = t1
+    oracle.set_threads(all_cores)
     return done, elapsed, cores
 
 
@@ -313,7 +316,8 @@ def combine_bytes(spec):
 
 def time_layer(spec, inp, b, steps, warmup, stream, flush):
     """Per-stage device times (ms, one row per step) through the per-stage
-    C-ABI calls, with L2 flushed before every step."""
+    C-ABI calls, with L2 flushed before every step (flush=None: warm L2, the
+    previous step's data left in it)."""
     import numpy as np
     import torch
     from combine_softmax_top_b200 import moe
@@ -339,18 +343,65 @@ def time_layer(spec, inp, b, steps, warmup, stream, flush):
             ev[4].record(stream)
 
     for _ in range(max(3, warmup)):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         step()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
     rc = moe.moe_poll_status(b.ws, stream)
     if rc != 0:
         raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
     return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)])
+
+
+def time_whole_layer(spec, inp, b, steps, warmup, flush):
+    """Whole-layer device time (ms per step) through the public moe_layer call:
+    stream-launched, and as the replay of a CUDA graph holding one call. L2 is
+    flushed before every timed step; the workspace's epoch protocol needs no
+    host work between replays."""
+    import numpy as np
+    import torch
+    from combine_softmax_top_b200 import moe
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        moe.run_layer(b, inp)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+
+    stream_ms = timed(lambda: moe.run_layer(b, inp))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        moe.run_layer(b, inp)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        moe.run_layer(b, inp)
+    for _ in range(3):
+        flush.zero_()
+        g.replay()
+    graph_ms = timed(g.replay)
+    rc = moe.moe_poll_status(b.ws)
+    del g
+    if rc != 0:
+        raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
+    return stream_ms, graph_ms
 
 
 def run_report(args):
@@ -379,6 +430,13 @@ def run_report(args):
                 "stage_us": {k: float(v * 1e3) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], st)},
                 "peak_source": kind}
         rb, db, cb = route_bytes(spec), dispatch_bytes(spec), combine_bytes(spec)
+        warm = time_layer(spec, inp, b, args.steps, args.warmup, stream, None).mean(0)
+        line["stage_us_warm_l2"] = {k: float(v * 1e3) for k, v in
+                                    zip(["route", "dispatch", "grouped_ffn", "combine"], warm)}
+        whole_ms, graph_ms = time_whole_layer(spec, inp, b, args.steps, args.warmup, flush)
+        line["layer_call_us"] = whole_ms * 1e3         # one moe_layer call, stream-launched
+        line["layer_graph_us"] = graph_ms * 1e3        # the same call replayed from a CUDA graph
+        line["graph_tokens_per_s"] = spec.T / (graph_ms / 1e3)
         line["route_GBps"] = rb / (st[0] / 1e3) / 1e9
         line["dispatch_GBps"] = db / (st[1] / 1e3) / 1e9
         line["combine_GBps"] = cb / (st[3] / 1e3) / 1e9
@@ -505,6 +563,15 @@ def run_ours(args):
                "h2d_bytes_per_step": hx.numel() * hx.element_size() + hl.numel() * hl.element_size(),
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
 
+    # the whole layer through one moe_layer call, stream-launched and replayed
+    # from a CUDA graph (outside the timed region above; reported beside it)
+    call_ms, graph_ms = time_whole_layer(spec, inp, b, args.steps, args.warmup, flush)
+    call_ms = max_over_ranks(call_ms, dev)
+    graph_ms = max_over_ranks(graph_ms, dev)
+    graph = {"us_per_layer": graph_ms * 1000.0, "value": job_throughput(spec.T, world, graph_ms),
+             "unit": "tokens/s", "stream_launched_us_per_layer": call_ms * 1000.0,
+             "how": "one moe_layer call captured in a CUDA graph; median replay, L2 flushed before each"}
+
     counts = b.counts.cpu().numpy()
     peaks, peak_kind = load_peaks()
     ffn_ms = float(stage[:, 2].mean())
@@ -536,6 +603,10 @@ def run_ours(args):
         n, el, cores = oracle_sample(spec, inp, args.cpu_seconds)
         cpu = {"value": n / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"first {n} of {spec.T} tokens of the same workload ({el:.1f}s)"}
+        if spec.name in ("tiny", "decode"):   # the same on one core
+            n1, el1, _ = oracle_sample(spec, inp, min(args.cpu_seconds, 10.0), threads=1)
+            cpu["one_core"] = {"value": n1 / el1, "unit": "tokens/s", "cores": 1,
+                               "sample": f"first {n1} of {spec.T} tokens ({el1:.1f}s)"}
 
     if rank == 0:
         line = {
@@ -555,6 +626,7 @@ def run_ours(args):
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "graph_replay": graph,
             "gpu_launches": args.steps * moe.kernels_per_layer(spec),
             "clocks": clk,
         }

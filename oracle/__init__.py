@@ -57,12 +57,19 @@ def lib() -> ctypes.CDLL:
             "oracle_expert_rows": [P, I64, P, P, P, P, P, P],
             "oracle_combine": [I64, I64, I64, I32, P, P, I32, P],
             "oracle_moe_layer": [P, P, P, I64, I64, P, P, P, P, P, P],
+            "oracle_set_threads": [I32],
         }
         for name, args in sigs.items():
             fn = getattr(_lib, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
     return _lib
+
+
+def set_threads(n: int) -> int:
+    """Limit the oracle's OpenMP loops to n threads (timing only); returns the
+    count in force."""
+    return int(lib().oracle_set_threads(int(n)))
 
 
 class OracleError(RuntimeError):

@@ -39,6 +39,9 @@
 #include <cstring>
 #include <vector>
 #include <algorithm>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 extern "C" {
 
@@ -453,6 +456,18 @@ int oracle_moe_layer(const oracle_problem* p, const void* x, const float* logits
     }
   }
   return ORC_OK;
+}
+
+// Threads the OpenMP loops use from now on (n >= 1); returns the count in
+// force. Timing aid only: the results do not depend on it.
+int oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+  return omp_get_max_threads();
+#else
+  (void)n;
+  return 1;
+#endif
 }
 
 }  // extern "C"
