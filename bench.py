@@ -421,14 +421,17 @@ def run_report(args):
     for spec in cases:
         inp = W.make_inputs(spec, seed=args.seed, device=dev)
         b = moe.alloc_buffers(spec, device=dev)
+        clocks = ClockSampler(0)
+        clocks.start()
         st = time_layer(spec, inp, b, args.steps, args.warmup, stream, flush).mean(0)
+        clk = clocks.stop()
         counts = b.counts.cpu().numpy()
         layer_ms = float(st.sum())
         line = {"report": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k,
                 "I": None if spec.identity else spec.I, "dtype": spec.weight if not spec.identity else spec.xq,
                 "layer_us": layer_ms * 1e3, "tokens_per_s": spec.T / (layer_ms / 1e3),
                 "stage_us": {k: float(v * 1e3) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], st)},
-                "peak_source": kind}
+                "peak_source": kind, "clocks": clk}
         rb, db, cb = route_bytes(spec), dispatch_bytes(spec), combine_bytes(spec)
         warm = time_layer(spec, inp, b, args.steps, args.warmup, stream, None).mean(0)
         line["stage_us_warm_l2"] = {k: float(v * 1e3) for k, v in

@@ -68,7 +68,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColSfa0 = 256, kColSfa1 = 260, kColSfb0 = 264;
 
 enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
-enum : int { kFfnGen = 3, kFfnExit = 4 };   // counter-set misc slots used here
+// counter-set misc slots used here: FFN calls completed on this dispatch, CTAs
+// that left the current call, the next unit to hand out
+enum : int { kFfnGen = 3, kFfnExit = 4, kFfnNext = 5 };
 
 struct TcParams {
   CUtensorMap tm_wg, tm_wu, tm_wd;
@@ -261,9 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   if (warp == kSchedWarp) {
     // ---------------------------------------------------------------- scheduler
     // Units, expert-major: for each expert, for each 128-feature slice, every
-    // tile of that expert (all gate/up units before all down units), dealt
-    // round-robin to the CTAs. Neighbouring CTAs thus work on the tiles of one
-    // expert with the same weight slice at the same time and share it in L2.
+    // tile of that expert (all gate/up units before all down units), handed
+    // out in that order from one global counter, so that CTAs that finish
+    // early take more units. CTAs working at the same time thus hold the tiles
+    // of one expert with the same weight slice and share it in L2.
     // For each unit the scheduler waits for the tile's sentinel (and a down
     // unit's h), splits the tile into chunks of <= kBRows rows and queues them.
     int* tile_pre = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1] first tile of each expert
@@ -309,7 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         *abort_flag = 1;
         good = false;
       }
-      for (uint32_t u = blockIdx.x; good && u < total; u += gridDim.x) {
+      // units are taken from one counter in increasing order (dynamic load
+      // balance); every unit waits only on units earlier in that order
+      while (good) {
+        const uint32_t u = atomicAdd(misc + kFfnNext, 1u);
+        if (u >= total) break;
         Job j;
         j.kind = u >= n1 ? kKindDown : kKindGateUp;
         const uint32_t v = j.kind == kKindDown ? u - n1 : u;
@@ -804,7 +811,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // the last CTA out records that one more FFN call ran on this dispatch
     __threadfence();
     const uint32_t exits = atomicAdd(misc + kFfnExit, 1u) + 1u;
-    if (exits == gridDim.x * (gen + 1u)) st_release(misc + kFfnGen, gen + 1u);
+    if (exits == gridDim.x * (gen + 1u)) {   // every CTA is done with the unit counter
+      misc[kFfnNext] = 0u;
+      __threadfence();
+      st_release(misc + kFfnGen, gen + 1u);
+    }
   }
 }
 
