@@ -163,6 +163,8 @@ cudaError_t launch_combine(const Ctx& c, const moe_dispatch_bufs& b, const void*
     row_dt = c.s.y_dtype;
   }
   if (a.T == 0) return cudaSuccess;
+  cudaError_t staged_err;
+  if (launch_combine_tma(c, b, y, topk_w, out, &staged_err)) return staged_err;
   const int64_t units = (int64_t)a.T * ((a.H + kChunk - 1) / kChunk);
   const int64_t want = (units + kWarps - 1) / kWarps;
   const int grid = (int)std::min<int64_t>(want, (int64_t)c.num_sms * 4);

@@ -213,6 +213,10 @@ cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float*
 // write_sf: also write the e4m3 scale atoms the tensor-core FFN reads
 cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
                             const moe_dispatch_bufs& b, bool write_sf = true);
+// The shared-memory-staged combine for many-token layers; false when the
+// shape does not suit it (nothing launched), else *err holds the launch result.
+bool launch_combine_tma(const Ctx& c, const moe_dispatch_bufs& b, const void* y, const float* topk_w, void* out,
+                        cudaError_t* err);
 cudaError_t launch_combine(const Ctx& c, const moe_dispatch_bufs& b, const void* y,
                            const float* topk_w, void* out);
 cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,

@@ -1,7 +1,9 @@
 """The whole layer through the C ABI on shapes off the five workloads: ragged
 tails, a single token, no tokens, k = 1, a hidden size whose K loop crosses 64
-scale blocks, and routing skewed so one expert's window spans several tiles
-(split into chunks by the tensor-core FFN)."""
+scale blocks, routing skewed so one expert's window spans several tiles
+(split into chunks by the tensor-core FFN), and layers with more than 32 rows
+per expert, whose tensor-core FFN uses 128-row tiles (down jobs over pairs of
+H slices when H/128 is even, single slices when it is odd)."""
 import numpy as np
 import pytest
 import torch
@@ -23,6 +25,10 @@ CASES = [
     ("long_k_fp8", "decode", dict(T=16, H=8320, E=4, k=2, I=256), 0.0),
     ("hot_expert_fp8", "decode", dict(T=256, H=512, E=64, k=2, I=256), 30.0),
     ("hot_expert_bf16", "skew", dict(T=256, H=256, E=64, k=2, I=256, zipf_s=0.0), 30.0),
+    # > 32 rows per expert: 128-row token tiles; ragged last tiles
+    ("big_tiles_pairs_fp8", "decode", dict(T=300, H=512, E=4, k=2, I=384), 0.0),     # H/128 even: down pairs
+    ("big_tiles_odd_h_fp8", "decode", dict(T=300, H=384, E=4, k=2, I=256), 0.0),     # H/128 odd: single slices
+    ("big_tiles_pairs_bf16", "skew", dict(T=260, H=256, E=4, k=2, I=256, zipf_s=0.0), 0.0),
     ("tiny_no_renorm", "tiny", dict(renorm=0), 0.0),
     ("fp32_ragged", "tiny", dict(T=45, H=384, E=7, k=3, I=256), 0.0),
 ]
