@@ -10,8 +10,9 @@
 // abstract).
 //
 // CTAs walk tokens; for each token:
-//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j (issued
-//     while the previous token's rows are being written);
+//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j (the
+//     expert index loaded two tokens ahead, the atomic issued one token
+//     ahead, so neither round trip stalls the CTA);
 //  2. all warps stream the token row once (16-byte loads) and write it to the
 //     k claimed rows; E4M3 rows are quantised per 128 values with the
 //     smallest power-of-two scale that keeps the block within +-448, and the
@@ -43,6 +44,45 @@ struct Args {
   int64_t set_words;
 };
 
+// Raw bytes of 16 consecutive values of x (bf16: 2 vectors, f32: 4).
+template <int kAct>
+struct Raw16 {
+  uint4 r[kAct == MOE_BF16 ? 2 : 4];
+};
+
+template <int kAct>
+__device__ __forceinline__ void load_raw(const void* x, int64_t off, Raw16<kAct>& v) {
+  if constexpr (kAct == MOE_BF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + off);
+    v.r[0] = __ldg(p);
+    v.r[1] = __ldg(p + 1);
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(x) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v.r[i] = __ldg(p + i);
+  }
+}
+
+template <int kAct>
+__device__ __forceinline__ void raw_to_f32(const Raw16<kAct>& v, float* f) {
+  if constexpr (kAct == MOE_BF16) {
+    const uint32_t w[8] = {v.r[0].x, v.r[0].y, v.r[0].z, v.r[0].w, v.r[1].x, v.r[1].y, v.r[1].z, v.r[1].w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[4 * i] = __uint_as_float(v.r[i].x);
+      f[4 * i + 1] = __uint_as_float(v.r[i].y);
+      f[4 * i + 2] = __uint_as_float(v.r[i].z);
+      f[4 * i + 3] = __uint_as_float(v.r[i].w);
+    }
+  }
+}
+
 __device__ __forceinline__ void load16(const void* x, int act, int64_t off, float* v) {
   if (act == MOE_BF16) {
     const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + off);
@@ -71,16 +111,23 @@ __device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e
                ((unsigned long long)epoch << 32) | ((unsigned long long)e << 16) | (unsigned)tile);
 }
 
-// Claim rows for the k slots of token t (threads tid < k); rows land in
-// s_row / s_e.
-__device__ __forceinline__ void claim_rows(const Args& a, int t, int tid, uint32_t* count, int* s_row,
-                                           int* s_e) {
-  if (tid >= a.k) return;
+// Row claims are pipelined over three tokens by the threads tid < k (slot
+// tid): the expert index is loaded two tokens ahead, the atomicAdd on its
+// count issued one token ahead, and its result used a whole token later, so
+// neither round trip stalls the CTA.
+__device__ __forceinline__ int load_expert(const Args& a, int t, int tid) {
+  return t < a.T ? __ldg(a.idx + (int64_t)t * a.k + tid) : -1;
+}
+
+__device__ __forceinline__ uint32_t issue_claim(const Args& a, int t, int e, uint32_t* count) {
+  return (t < a.T && e >= 0 && e < a.E) ? atomicAdd(count + e, 1u) : 0u;
+}
+
+// Token t's slot tid: the claimed row (or -1), recorded in pos/row_src/s_row.
+__device__ __forceinline__ void finish_claim(const Args& a, int t, int tid, int e, uint32_t p, int* s_row, int* s_e) {
   const int pair = t * a.k + tid;
-  const int e = __ldg(a.idx + pair);
   int row = -1;
   if (e >= 0 && e < a.E) {
-    const uint32_t p = atomicAdd(count + e, 1u);
     if (p < (uint32_t)a.cap) {
       row = e * a.cap + (int)p;
       a.b.row_src[row] = pair;
@@ -96,22 +143,15 @@ __device__ __forceinline__ void claim_rows(const Args& a, int t, int tid, uint32
 }
 
 // Write token t's row to its claimed rows (all threads; a lane group of 8
-// covers one 128-value block). v0 holds this thread's first slice.
-__device__ __forceinline__ void stream_row(const Args& a, int t, int tid, const int* s_row, const float* v0) {
-  const int steps = a.H / kElems;
-  for (int s = tid; s < (steps + 31) / 32 * 32; s += kThreads) {
-    const bool live = s < steps;
+// covers one 128-value block). pre holds this thread's first kPre slices
+// (loaded one token ahead); further slices (H > kPre * 4096) load here.
+constexpr int kPre = 2;
+
+// Quantise (or convert) one 16-value slice s of token t and store it to the
+// token's k rows; all lanes of the warp take part (the 8-lane amax).
+__device__ __forceinline__ void put_slice(const Args& a, int tid, const int* s_row, int s, bool live, const float* v) {
+  {
     const int h0 = s * kElems;
-    float v[kElems];
-    if (live && s == tid) {
-#pragma unroll
-      for (int i = 0; i < kElems; ++i) v[i] = v0[i];
-    } else if (live) {
-      load16(a.x, a.act, (int64_t)t * a.H + h0, v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < kElems; ++i) v[i] = 0.f;
-    }
     if (a.xq_dtype == MOE_E4M3) {
       float amax = 0.f;
 #pragma unroll
@@ -119,7 +159,7 @@ __device__ __forceinline__ void stream_row(const Args& a, int t, int tid, const 
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-      if (!live) continue;
+      if (!live) return;
       const int p = pow2_scale_exp(amax);
       const float inv = exp2i(-p > -126 ? -p : -126);  // 2^-p; p <= 120 for finite x
       uint32_t q[4];
@@ -168,6 +208,34 @@ __device__ __forceinline__ void stream_row(const Args& a, int t, int tid, const 
   }
 }
 
+template <int kAct>
+__device__ __forceinline__ void stream_row(const Args& a, int t, int tid, const int* s_row, const Raw16<kAct>* pre) {
+  const int steps = a.H / kElems;
+  const int span = (steps + 31) / 32 * 32;   // whole warps take part in every pass
+#pragma unroll
+  for (int si = 0; si < kPre; ++si) {
+    const int s = tid + si * kThreads;
+    if (s >= span) break;
+    float v[kElems];
+    if (s < steps) raw_to_f32<kAct>(pre[si], v);
+    else {
+#pragma unroll
+      for (int i = 0; i < kElems; ++i) v[i] = 0.f;
+    }
+    put_slice(a, tid, s_row, s, s < steps, v);
+  }
+  for (int s = tid + kPre * kThreads; s < span; s += kThreads) {
+    float v[kElems];
+    if (s < steps) load16(a.x, a.act, (int64_t)t * a.H + s * kElems, v);
+    else {
+#pragma unroll
+      for (int i = 0; i < kElems; ++i) v[i] = 0.f;
+    }
+    put_slice(a, tid, s_row, s, s < steps, v);
+  }
+}
+
+template <int kAct>
 __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
   __shared__ int s_row[2][kMaxTopk];   // double-buffered: this token's rows, the next token's
   __shared__ int s_e[2][kMaxTopk];
@@ -192,26 +260,45 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     for (int64_t i = lo + tid; i < hi; i += kThreads) next[i] = 0u;
   }
 
-  // Tokens blockIdx.x, + gridDim.x, ...: the next token's first row slice and
-  // row claims are issued before this token's rows are written, so their
-  // round trips overlap the streaming.
+  // Tokens blockIdx.x, + G, + 2G, ... (G = gridDim.x). The next token's row
+  // slices are loaded while this token is written, and its row claims were
+  // issued a token earlier still.
+  const int G = gridDim.x;
   const int steps = a.H / kElems;
   int cur = 0;
   int t = blockIdx.x;
-  float v0[kElems];
+  Raw16<kAct> v0[kPre];
+  int e1 = -1, e2 = -1;   // slot tid's expert for tokens t + G and t + 2G
+  uint32_t p1 = 0;        // and the claim already issued for token t + G
+  if (tid < a.k && t < a.T) {
+    const int e0 = load_expert(a, t, tid);
+    const uint32_t p0 = issue_claim(a, t, e0, count);
+    e1 = load_expert(a, t + G, tid);
+    p1 = issue_claim(a, t + G, e1, count);
+    e2 = load_expert(a, t + 2 * G, tid);
+    finish_claim(a, t, tid, e0, p0, s_row[0], s_e[0]);
+  }
   if (t < a.T) {
-    if (tid < steps) load16(a.x, a.act, (int64_t)t * a.H + tid * kElems, v0);
-    claim_rows(a, t, tid, count, s_row[0], s_e[0]);
+#pragma unroll
+    for (int i = 0; i < kPre; ++i)
+      if (tid + i * kThreads < steps) load_raw<kAct>(a.x, (int64_t)t * a.H + (tid + i * kThreads) * kElems, v0[i]);
   }
   __syncthreads();
-  for (; t < a.T; t += gridDim.x) {
-    const int tn = t + gridDim.x;
-    float vn[kElems];
-    if (tn < a.T) {
-      if (tid < steps) load16(a.x, a.act, (int64_t)tn * a.H + tid * kElems, vn);
-      claim_rows(a, tn, tid, count, s_row[cur ^ 1], s_e[cur ^ 1]);
+  for (; t < a.T; t += G) {
+    const int tn = t + G;
+    if (tid < a.k && tn < a.T) {
+      finish_claim(a, tn, tid, e1, p1, s_row[cur ^ 1], s_e[cur ^ 1]);   // claimed a token ago
+      p1 = issue_claim(a, tn + G, e2, count);
+      e1 = e2;
+      e2 = load_expert(a, tn + 2 * G, tid);
     }
-    stream_row(a, t, tid, s_row[cur], v0);
+    Raw16<kAct> vn[kPre];
+    if (tn < a.T) {
+#pragma unroll
+      for (int i = 0; i < kPre; ++i)
+        if (tid + i * kThreads < steps) load_raw<kAct>(a.x, (int64_t)tn * a.H + (tid + i * kThreads) * kElems, vn[i]);
+    }
+    stream_row<kAct>(a, t, tid, s_row[cur], v0);
     __threadfence();
     __syncthreads();
     // count the filled rows; the bump that completes a tile publishes it
@@ -226,7 +313,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
       }
     }
 #pragma unroll
-    for (int i = 0; i < kElems; ++i) v0[i] = vn[i];
+    for (int i = 0; i < kPre; ++i) v0[i] = vn[i];
     cur ^= 1;
     __syncthreads();   // the next token's claims are visible; this token's rows are free
   }
@@ -281,14 +368,18 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
   a.set_words = (int64_t)c.L.set_words;
   // one wave of resident CTAs, each walking several tokens (fewer CTAs also
   // means fewer arrivals on the closing counter)
-  static int resident = 0;
-  if (resident == 0) {
-    int r = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, dispatch_kernel, kThreads, 0) != cudaSuccess || r < 1) r = 1;
-    resident = r;
-  }
-  const int grid = a.T > 0 ? std::min(a.T, c.num_sms * resident) : 1;
-  dispatch_kernel<<<grid, kThreads, 0, c.stream>>>(a);
+  auto go = [&](auto kern, int& resident) {
+    if (resident == 0) {
+      int r = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kThreads, 0) != cudaSuccess || r < 1) r = 1;
+      resident = r;
+    }
+    const int grid = a.T > 0 ? std::min(a.T, c.num_sms * resident) : 1;
+    kern<<<grid, kThreads, 0, c.stream>>>(a);
+  };
+  static int resident_bf16 = 0, resident_f32 = 0;
+  if (a.act == MOE_BF16) go(dispatch_kernel<MOE_BF16>, resident_bf16);
+  else go(dispatch_kernel<MOE_F32>, resident_f32);
   return cudaGetLastError();
 }
 
