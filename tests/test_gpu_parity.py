@@ -273,3 +273,30 @@ def test_ffn_wait_runs_out_and_context_survives(cuda_device):
     p = G.oracle_problem(s, inp)
     r = oracle.moe_layer(p, raw(inp["x"]), raw(inp["logits"]))
     assert max_abs_rel(as_f64(raw(b2.out), "bf16"), as_f64(r["out"], "bf16")) < 2e-2
+
+
+@pytest.mark.parametrize("xq", ["e4m3", "bf16"])
+def test_staged_combine_with_dropped_rows(xq, cuda_device):
+    """Layers with many tokens take the shared-memory-staged combine; slots
+    whose row was dropped (capacity overflow, pos = -1) add nothing, and k = 3
+    exercises a slot count that is not a power of two."""
+    s = W.spec("sweep", T=1024, H=512, E=4, k=3, xq=xq, cap_rows=512)
+    inp = W.make_inputs(s, seed=3, device="cuda")
+    inp["logits"][:, 0] += 100.0              # every token picks expert 0 first: 512 of them kept
+    b = G.run_stages(s, inp)
+    assert G.poll(b) == 4                     # MOE_ERR_CAPACITY, reported; the layer still completes
+    pos = b.pos.cpu().numpy().astype(np.int64)
+    w = b.topk_w.cpu().numpy()
+    assert (pos.reshape(s.T, s.k)[:, 0] == -1).sum() == 512   # (the other experts overflow too)
+    keep = pos >= 0
+    safe = np.where(keep, pos, 0)
+    if xq == "e4m3":
+        rows = oracle.e4m3_decode(G.gather(b.xq, safe)) * np.repeat(G.gather(b.xs, safe).astype(np.float64), 128, axis=1)
+    else:
+        rows = values(G.gather(b.xq, safe), "bf16")
+    rows = np.where(keep[:, None], rows, 0.0).astype(np.float32)   # exact in fp32
+    out = oracle.combine(rows, w, oracle.F32, G.ODT[s.out])
+    got = raw(b.out)
+    mag = (np.abs(w.astype(np.float64)).reshape(-1, 1) * np.abs(rows.astype(np.float64))).reshape(s.T, s.k, -1).sum(1)
+    g, r = bf16_bits_to_f32(got).astype(np.float64), bf16_bits_to_f32(out).astype(np.float64)
+    assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 2 * s.k * 2.0 ** -24 * mag + 1e-30)
