@@ -121,11 +121,12 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
       float g[16], uu[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) { g[i] = 0.f; uu[i] = 0.f; }
-      for (int k0 = 0; k0 < K; k0 += kK) {
-        // every load of this K step is issued before any is used
-        constexpr int kXPer = kR * kK / kThreads;   // 4
-        constexpr int kWPer = kF * kK / kThreads;   // 16
-        float xv[kXPer], wv0[kWPer], wv1[kWPer];
+      // K steps software-pipelined: the next step's loads are issued before
+      // this step's FMAs, so each step's global-load latency overlaps work
+      constexpr int kXPer = kR * kK / kThreads;   // 4
+      constexpr int kWPer = kF * kK / kThreads;   // 16
+      float xv[kXPer], wv0[kWPer], wv1[kWPer], sc0 = 1.f, sc1 = 1.f;
+      auto load_step = [&](int k0) {
 #pragma unroll
         for (int i = 0; i < kXPer; ++i) {
           const int idx = tid + kThreads * i, r = idx / kK, kk = idx % kK;
@@ -136,7 +137,6 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
             if (xdt == MOE_E4M3) xv[i] *= xsc[row * (K / kQBlock) + (k0 + kk) / kQBlock];
           }
         }
-        float sc0 = 1.f, sc1 = 1.f;
         if (a.w_dt == MOE_E4M3) {
           const int64_t sidx = ((int64_t)e * (NF / kQBlock) + f0 / kQBlock) * (K / kQBlock) + k0 / kQBlock;
           sc0 = s0[sidx];
@@ -149,6 +149,9 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
           wv0[i] = ld_act(w0, a.w_dt, widx);
           wv1[i] = DOWN ? 0.f : ld_act(w1, a.w_dt, widx);
         }
+      };
+      load_step(0);
+      for (int k0 = 0; k0 < K; k0 += kK) {
 #pragma unroll
         for (int i = 0; i < kXPer; ++i) {
           const int idx = tid + kThreads * i;
@@ -161,15 +164,16 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
           if (!DOWN) sw1[idx / kK][idx % kK] = wv1[i] * sc1;
         }
         __syncthreads();
+        if (k0 + kK < K) load_step(k0 + kK);
 #pragma unroll 4
         for (int kk = 0; kk < kK; ++kk) {
           const float b0 = sw0[f][kk];
           const float b1 = DOWN ? 0.f : sw1[f][kk];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float xv = sx[rh * 16 + i][kk];
-            g[i] = fmaf(xv, b0, g[i]);
-            if (!DOWN) uu[i] = fmaf(xv, b1, uu[i]);
+            const float xv_ = sx[rh * 16 + i][kk];
+            g[i] = fmaf(xv_, b0, g[i]);
+            if (!DOWN) uu[i] = fmaf(xv_, b1, uu[i]);
           }
         }
         __syncthreads();
