@@ -300,3 +300,31 @@ def test_staged_combine_with_dropped_rows(xq, cuda_device):
     mag = (np.abs(w.astype(np.float64)).reshape(-1, 1) * np.abs(rows.astype(np.float64))).reshape(s.T, s.k, -1).sum(1)
     g, r = bf16_bits_to_f32(got).astype(np.float64), bf16_bits_to_f32(out).astype(np.float64)
     assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 2 * s.k * 2.0 ** -24 * mag + 1e-30)
+
+
+@pytest.mark.parametrize("over", [dict(T=64, H=512, E=8, k=2, I=256),        # 64-row tiles
+                                  dict(T=300, H=512, E=4, k=2, I=384)],      # 128-row tiles, down pairs
+                         ids=["small_tiles", "big_tiles"])
+def test_ffn_repeated_on_one_dispatch(over, cuda_device):
+    """The grouped FFN run three times on one dispatch: each call hands out its
+    units from a counter that the call's last CTA resets, and counts its calls
+    for the down units' dependency; every call must give the same bits."""
+    s = W.spec("decode", **over)
+    inp = W.make_inputs(s, seed=5, device="cuda")
+    b = moe.alloc_buffers(s)
+    bufs = b.dispatch_bufs()
+    w = moe.weights_struct(inp)
+    moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws)
+    moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, bufs)
+    ys, hs = [], []
+    for _ in range(3):
+        b.y.zero_()
+        b.hq.view(torch.uint8).zero_()
+        moe.moe_grouped_ffn(b.shape, bufs, w, b.ws, b.y)
+        torch.cuda.synchronize()
+        assert G.poll(b) == 0
+        ys.append(b.y.clone())
+        hs.append(b.hq.view(torch.uint8).clone())
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    assert torch.equal(hs[0], hs[1]) and torch.equal(hs[1], hs[2])
+    assert ys[0].abs().sum().item() > 0
