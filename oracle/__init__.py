@@ -98,7 +98,7 @@ class _Problem(ctypes.Structure):
         ("x_dtype", ctypes.c_int32), ("xq_dtype", ctypes.c_int32),
         ("w_dtype", ctypes.c_int32), ("h_dtype", ctypes.c_int32),
         ("y_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-        ("renorm", ctypes.c_int32), ("identity", ctypes.c_int32),
+        ("renorm", ctypes.c_int32), ("identity", ctypes.c_int32), ("shared", ctypes.c_int32),
         ("w_gate", ctypes.POINTER(ctypes.c_void_p)), ("w_up", ctypes.POINTER(ctypes.c_void_p)),
         ("w_down", ctypes.POINTER(ctypes.c_void_p)),
         ("s_gate", ctypes.POINTER(ctypes.c_void_p)), ("s_up", ctypes.POINTER(ctypes.c_void_p)),
@@ -114,18 +114,21 @@ class Problem:
 
     Weights are either full arrays ([E, I, H] gate/up, [E, H, I] down, e4m3
     scales [E, I/128, H/128] / [E, H/128, I/128]) or mappings from expert index
-    to that expert's matrix, for checks that touch only a few experts.
+    to that expert's matrix, for checks that touch only a few experts. With
+    shared=1 the arrays hold E + 1 experts: expert E is the shared expert that
+    every token also goes through, added with weight 1.
     """
 
     def __init__(self, T, H, E, k, I, *, x_dtype, xq_dtype, w_dtype, h_dtype, y_dtype,
-                 out_dtype, renorm=1, identity=0, w_gate: ExpertWeights = None,
+                 out_dtype, renorm=1, identity=0, shared=0, w_gate: ExpertWeights = None,
                  w_up: ExpertWeights = None, w_down: ExpertWeights = None,
                  s_gate: ExpertWeights = None, s_up: ExpertWeights = None,
                  s_down: ExpertWeights = None):
         self.T, self.H, self.E, self.k, self.I = int(T), int(H), int(E), int(k), int(I)
         self.x_dtype, self.xq_dtype, self.w_dtype = x_dtype, xq_dtype, w_dtype
         self.h_dtype, self.y_dtype, self.out_dtype = h_dtype, y_dtype, out_dtype
-        self.renorm, self.identity = int(renorm), int(identity)
+        self.renorm, self.identity, self.shared = int(renorm), int(identity), int(shared)
+        self.nw = self.E + self.shared     # experts with weights
         self._keep = []
         tabs = []
         for w in (w_gate, w_up, w_down, s_gate, s_up, s_down):
@@ -134,18 +137,18 @@ class Problem:
         s.T, s.H, s.E, s.k, s.I = self.T, self.H, self.E, self.k, self.I
         s.x_dtype, s.xq_dtype, s.w_dtype = x_dtype, xq_dtype, w_dtype
         s.h_dtype, s.y_dtype, s.out_dtype = h_dtype, y_dtype, out_dtype
-        s.renorm, s.identity = self.renorm, self.identity
+        s.renorm, s.identity, s.shared = self.renorm, self.identity, self.shared
         s.w_gate, s.w_up, s.w_down, s.s_gate, s.s_up, s.s_down = tabs
         self._s = s
 
     def _table(self, w: ExpertWeights):
-        arr = (ctypes.c_void_p * self.E)()
+        arr = (ctypes.c_void_p * self.nw)()
         if w is None:
             pass
         elif isinstance(w, np.ndarray):
-            assert w.shape[0] == self.E and w.flags["C_CONTIGUOUS"]
+            assert w.shape[0] == self.nw and w.flags["C_CONTIGUOUS"]
             self._keep.append(w)
-            for e in range(self.E):
+            for e in range(self.nw):
                 arr[e] = w[e].ctypes.data
         else:
             for e, m in w.items():
@@ -247,8 +250,9 @@ def combine(y_pairs: np.ndarray, w: np.ndarray, y_dtype: int, out_dtype: int) ->
 
 def moe_layer(p: Problem, x: np.ndarray, logits: np.ndarray, t0: int = 0, t1: int | None = None,
               want_intermediates: bool = False):
-    """Whole layer for tokens [t0, t1). Returns dict with idx, w, out (and
-    xq, xs, y_pairs when want_intermediates)."""
+    """Whole layer for tokens [t0, t1). Returns dict with idx, w (the k routed
+    slots), out (and xq, xs, y_pairs when want_intermediates; y_pairs has
+    k + shared rows per token, the shared expert's last)."""
     t1 = p.T if t1 is None else t1
     n = t1 - t0
     x = np.ascontiguousarray(x)
@@ -260,7 +264,7 @@ def moe_layer(p: Problem, x: np.ndarray, logits: np.ndarray, t0: int = 0, t1: in
     if want_intermediates:
         xq = np.empty((n, p.H), _NP[p.xq_dtype])
         xs = np.empty((n, p.H // 128), np.float32) if p.xq_dtype == E4M3 else None
-        yp = None if p.identity else np.empty((n * p.k, p.H), _NP[p.y_dtype])
+        yp = None if p.identity else np.empty((n * (p.k + p.shared), p.H), _NP[p.y_dtype])
     _call("oracle_moe_layer", p.ref, _ptr(x), _ptr(logits), t0, t1, _ptr(idx), _ptr(w),
           _ptr(out), _ptr(xq), _ptr(xs), _ptr(yp))
     res = {"idx": idx, "w": w, "out": out}

@@ -64,7 +64,9 @@ typedef struct oracle_problem {
   int32_t out_dtype;  // ORC_F32 or ORC_BF16: layer output
   int32_t renorm;     // 1: weights renormalised over the k selected experts
   int32_t identity;   // 1: every expert is the identity map on its input
-  // One pointer per expert (E entries each). Expert e's matrices are
+  int32_t shared;     // 1: expert E is a shared expert every token also goes
+                      //    through, added with weight 1 after the k routed ones
+  // One pointer per expert (E + shared entries each). Expert e's matrices are
   // row-major: gate/up [I, H], down [H, I]; e4m3 scales [I/128, H/128] and
   // [H/128, I/128]. A NULL entry marks an expert whose weights were not
   // provided; using it is an error.
@@ -266,7 +268,7 @@ static inline double weight_at(const void* w, const float* s, int32_t dt,
 }
 
 static bool have_expert(const oracle_problem* p, int64_t e) {
-  if (e < 0 || e >= p->E) return false;
+  if (e < 0 || e >= p->E + (p->shared ? 1 : 0)) return false;
   if (!p->w_gate[e] || !p->w_up[e] || !p->w_down[e]) return false;
   if (p->w_dtype == ORC_E4M3 && (!p->s_gate[e] || !p->s_up[e] || !p->s_down[e])) return false;
   return true;
@@ -361,6 +363,7 @@ static int64_t dtype_bytes(int32_t dt) { return dt == ORC_F32 ? 4 : dt == ORC_BF
 static int check_problem(const oracle_problem* p) {
   if (!p || p->T < 0 || p->H <= 0 || p->E <= 0 || p->k <= 0 || p->k > p->E || p->I <= 0)
     return ORC_BAD_ARG;
+  if (p->shared != 0 && p->shared != 1) return ORC_BAD_ARG;
   if (p->xq_dtype == ORC_E4M3 && p->H % 128) return ORC_BAD_ARG;
   if (p->h_dtype == ORC_E4M3 && p->I % 128) return ORC_BAD_ARG;
   if (p->w_dtype == ORC_E4M3 && (p->H % 128 || p->I % 128)) return ORC_BAD_ARG;
@@ -428,26 +431,31 @@ int oracle_moe_layer(const oracle_problem* p, const void* x, const float* logits
   rc = oracle_route(p->T, p->E, p->k, p->renorm, logits, idx, w);
   if (rc) return rc;
   const int64_t H = p->H, k = p->k;
+  // slots per token: the k routed experts, then the shared expert E (weight 1)
+  const int64_t ks = k + (p->shared ? 1 : 0);
   const int64_t qb = dtype_bytes(p->xq_dtype), yb = dtype_bytes(p->y_dtype);
-  if (!p->identity)
+  if (!p->identity) {
     for (int64_t t = t0; t < t1; ++t)
       for (int64_t j = 0; j < k; ++j)
         if (!have_expert(p, idx[t * k + j])) return ORC_BAD_ARG;
+    if (p->shared && !have_expert(p, p->E)) return ORC_BAD_ARG;
+  }
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t t = t0; t < t1; ++t) {
     const int64_t lt = t - t0;
     std::vector<double> xh(H), yd(H), acc(H, 0.0);
     token_input(p, x, t, xh.data(), xq_tok ? (char*)xq_tok + lt * H * qb : nullptr,
                 xs_tok ? xs_tok + lt * (H / 128) : nullptr);
-    for (int64_t j = 0; j < k; ++j) {
-      const int64_t e = idx[t * k + j];
-      void* yrow = y_pair ? (char*)y_pair + (lt * k + j) * H * yb : nullptr;
+    for (int64_t j = 0; j < ks; ++j) {
+      const int64_t e = j < k ? idx[t * k + j] : p->E;
+      const double wj = j < k ? (double)w[t * k + j] : 1.0;
+      void* yrow = y_pair ? (char*)y_pair + (lt * ks + j) * H * yb : nullptr;
       if (p->identity) {
         for (int64_t c = 0; c < H; ++c) yd[c] = xh[c];
       } else {
         expert_row(p, e, xh.data(), nullptr, nullptr, yrow, yd.data());
       }
-      for (int64_t c = 0; c < H; ++c) acc[c] += (double)w[t * k + j] * yd[c];
+      for (int64_t c = 0; c < H; ++c) acc[c] += wj * yd[c];
     }
     for (int64_t c = 0; c < H; ++c) {
       float a32 = (float)acc[c];

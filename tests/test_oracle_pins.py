@@ -424,3 +424,48 @@ def test_missing_expert_weights_is_an_error():
                        w_up={0: raw(inp["w_up"][0])}, w_down={0: raw(inp["w_down"][0])})
     with pytest.raises(oracle.OracleError):
         oracle.expert_rows(p, np.array([1], np.int32), raw(inp["x"][:1]))
+
+
+def _shared_problem(s, wg, wu, wd, shared):
+    return oracle.Problem(s.T, s.H, s.E, s.k, s.I, x_dtype=oracle.F32, xq_dtype=oracle.F32,
+                          w_dtype=oracle.F32, h_dtype=oracle.F32, y_dtype=oracle.F32,
+                          out_dtype=oracle.F32, renorm=1, shared=shared, w_gate=raw(wg), w_up=raw(wu),
+                          w_down=raw(wd))
+
+
+def test_zero_shared_expert_changes_nothing():
+    """A shared expert with all-zero weights adds exactly zero: the layer equals
+    the one without it, bit for bit."""
+    s = W.spec("tiny")
+    inp = W.make_inputs(s, seed=6)
+    z = torch.zeros_like(inp["w_gate"][:1])
+    zd = torch.zeros_like(inp["w_down"][:1])
+    wg = torch.cat([inp["w_gate"], z]).contiguous()
+    wu = torch.cat([inp["w_up"], z]).contiguous()
+    wd = torch.cat([inp["w_down"], zd]).contiguous()
+    plain = oracle.moe_layer(_shared_problem(s, inp["w_gate"], inp["w_up"], inp["w_down"], 0),
+                             raw(inp["x"]), raw(inp["logits"]))
+    with_shared = oracle.moe_layer(_shared_problem(s, wg, wu, wd, 1), raw(inp["x"]), raw(inp["logits"]))
+    assert np.array_equal(plain["idx"], with_shared["idx"])
+    assert np.array_equal(plain["out"], with_shared["out"])
+
+
+def test_shared_expert_alone_is_the_dense_ffn():
+    """Routed experts with all-zero weights and a shared expert: the layer is
+    the shared expert's dense SwiGLU FFN of every token, whatever the routing."""
+    s = W.spec("tiny")
+    inp = W.make_inputs(s, seed=7)
+    E = s.E
+    z = torch.zeros_like(inp["w_gate"])
+    zd = torch.zeros_like(inp["w_down"])
+    wg = torch.cat([z, inp["w_gate"][:1]]).contiguous()
+    wu = torch.cat([z, inp["w_up"][:1]]).contiguous()
+    wd = torch.cat([zd, inp["w_down"][:1]]).contiguous()
+    r = oracle.moe_layer(_shared_problem(s, wg, wu, wd, 1), raw(inp["x"]), raw(inp["logits"]),
+                         want_intermediates=True)
+    _, ref = _dense_ffn_torch(inp["x"].double(), wg[E].double(), wu[E].double(), wd[E].double())
+    assert max_abs_rel(r["out"], ref.numpy()) < 1e-6
+    # the shared expert's row is the last of each token's k + 1 rows
+    yp = r["y_pairs"].reshape(s.T, s.k + 1, s.H)
+    assert max_abs_rel(yp[:, s.k], ref.numpy()) < 1e-6
+    assert np.all(yp[:, : s.k] == 0)
