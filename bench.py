@@ -37,6 +37,8 @@ def parse():
     p.add_argument("--config", default="decode")
     p.add_argument("--T", type=int, default=None, help="override the token count")
     p.add_argument("--E", type=int, default=None, help="override the expert count (small profiling cases)")
+    p.add_argument("--shared-expert", action="store_true",
+                   help="add one shared expert every token also goes through (weight 1)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -56,6 +58,8 @@ def overrides(args) -> dict:
         o["T"] = args.T
     if args.E:
         o["E"] = args.E
+    if getattr(args, "shared_expert", False):
+        o["shared"] = 1
     return o
 
 
@@ -177,6 +181,8 @@ def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None, thre
     logits = host(inp["logits"])
     x = host(inp["x"])
     idx, _ = oracle.route(logits, spec.k, spec.renorm)
+    if spec.shared:   # every token also goes through the shared expert E
+        idx = np.concatenate([idx, np.full((idx.shape[0], 1), spec.E, idx.dtype)], axis=1)
     limit = spec.T if max_tokens is None else min(spec.T, max_tokens)
     chunk = max(1, min(cores, limit))
     done = 0
@@ -189,7 +195,7 @@ def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None, thre
             for n in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
                 if inp.get(n) is not None:
                     kw[n] = {e: host(inp[n][e]) for e in experts}
-        p = oracle.Problem(spec.T, spec.H, spec.E, spec.k, spec.I, x_dtype=odt[spec.act],
+        p = oracle.Problem(spec.T, spec.H, spec.E, spec.k, spec.I, shared=spec.shared, x_dtype=odt[spec.act],
                            xq_dtype=odt[spec.xq], w_dtype=odt[spec.weight], h_dtype=odt[spec.h],
                            y_dtype=odt[spec.y], out_dtype=odt[spec.out], renorm=spec.renorm,
                            identity=spec.identity, **kw)
@@ -294,15 +300,16 @@ EL = {"f32": 4, "bf16": 2, "e4m3": 1}
 
 
 def route_bytes(spec):
-    return spec.T * (4 * spec.E + 8 * spec.k)
+    return spec.T * (4 * spec.E + 8 * spec.ks)
 
 
 def dispatch_bytes(spec):
-    """x read once, k rows (+ scales and scale atoms) written, pos/row_src."""
+    """x read once, k rows (+ scales and scale atoms) written, pos/row_src
+    (k + 1 slots with a shared expert)."""
     per_pair = spec.H * EL[spec.xq] + 8
     if spec.xq == "e4m3":
         per_pair += 2 * (spec.H // 128) * 4
-    return spec.T * (spec.H * EL[spec.act] + 4 * spec.k + spec.k * per_pair)
+    return spec.T * (spec.H * EL[spec.act] + 4 * spec.ks + spec.ks * per_pair)
 
 
 def combine_bytes(spec):
@@ -311,7 +318,7 @@ def combine_bytes(spec):
         row = spec.H * EL[spec.xq] + ((spec.H // 128) * 4 if spec.xq == "e4m3" else 0)
     else:
         row = spec.H * EL[spec.y]
-    return spec.T * (spec.k * (row + 8) + spec.H * EL[spec.out])
+    return spec.T * (spec.ks * (row + 8) + spec.H * EL[spec.out])
 
 
 def time_layer(spec, inp, b, steps, warmup, stream, flush):
@@ -416,7 +423,8 @@ def run_report(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     peaks, kind = load_peaks()
     hbm = peaks["hbm_gbs"]
-    cases = [W.spec("tiny"), W.spec("decode"), W.spec("prefill"), W.spec("skew")] + \
+    cases = [W.spec("tiny"), W.spec("decode"), W.spec("prefill"), W.spec("skew"),
+             W.spec("decode", shared=1), W.spec("prefill", shared=1)] + \
         [W.spec("sweep", T=t) for t in W.SWEEP_T]
     for spec in cases:
         inp = W.make_inputs(spec, seed=args.seed, device=dev)
@@ -427,7 +435,8 @@ def run_report(args):
         clk = clocks.stop()
         counts = b.counts.cpu().numpy()
         layer_ms = float(st.sum())
-        line = {"report": spec.name, "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k,
+        line = {"report": spec.name + ("+shared" if spec.shared else ""), "T": spec.T, "H": spec.H, "E": spec.E,
+                "topk": spec.k, "shared_experts": spec.shared,
                 "I": None if spec.identity else spec.I, "dtype": spec.weight if not spec.identity else spec.xq,
                 "layer_us": layer_ms * 1e3, "tokens_per_s": spec.T / (layer_ms / 1e3),
                 "stage_us": {k: float(v * 1e3) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], st)},
@@ -619,9 +628,9 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "e4m3" if spec.weight == "e4m3" else spec.weight,
             "data": "synthetic (seeded; random-init weights, no checkpoint)",
             "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
-                                   f"top-{spec.k} I={spec.I} "
+                                   f"top-{spec.k}{' + 1 shared expert' if spec.shared else ''} I={spec.I} "
                                    f"{'e4m3 128x128-block weights, bf16 tokens' if spec.weight == 'e4m3' else spec.weight}",
-                       "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I,
+                       "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I, "shared_experts": spec.shared,
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) before every timed step; weights 11 GB > L2"},
             "stage_us": {k: float(stage[:, j].mean() * 1000.0)

@@ -67,11 +67,14 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x
   if (st != MOE_OK) return st;
   if (shape->T > 0 && (!x || !topk_idx)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
-  st = check_bufs(shape, bufs, false);
-  if (st != MOE_OK) return st;
   Ctx c;
-  c.s = *shape;
-  c.L = make_layout(*shape);
+  c.s = effective_shape(*shape);
+  c.routed_E = shape->E;
+  c.routed_k = shape->topk;
+  c.shared = (shape->flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0;
+  st = check_bufs(&c.s, bufs, false);
+  if (st != MOE_OK) return st;
+  c.L = make_layout(c.s);
   // counters, sentinels and ring only: the scale atoms for the tensor-core
   // FFN are not written on this path
   if (c.L.off_xsf > kNoAllocScratchBytes) return MOE_ERR_INVALID_ARG;   // too big for the fixed scratch

@@ -19,7 +19,10 @@ moe_status check_shape(const moe_shape* s) {
   if (!s) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->H <= 0 || s->E < 1 || s->E > 65535) return MOE_ERR_INVALID_ARG;
   if (s->topk < 1 || s->topk > s->E || s->topk > kMaxTopk) return MOE_ERR_INVALID_ARG;
-  if (s->quant_block != kQBlock || s->flags != 0) return MOE_ERR_INVALID_ARG;
+  if (s->quant_block != kQBlock || (s->flags & ~MOE_FLAG_SHARED_EXPERT) != 0) return MOE_ERR_INVALID_ARG;
+  const bool shared = (s->flags & MOE_FLAG_SHARED_EXPERT) != 0;
+  if (shared && (s->identity_experts || s->topk + 1 > kMaxTopk || s->E + 1 > 65535 || default_cap(*s) < s->T))
+    return MOE_ERR_INVALID_ARG;   // the shared expert takes every token
   if ((s->renorm != 0 && s->renorm != 1) || (s->identity_experts != 0 && s->identity_experts != 1))
     return MOE_ERR_INVALID_ARG;
   if (s->cap_rows < 0 || (s->cap_rows > 0 && s->cap_rows % kTileRows != 0)) return MOE_ERR_INVALID_ARG;
@@ -30,8 +33,9 @@ moe_status check_shape(const moe_shape* s) {
   if (s->act_dtype == MOE_E4M3 || s->out_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (s->xq_dtype == MOE_E4M3 && s->H % kQBlock != 0) return MOE_ERR_INVALID_ARG;
   const int64_t cap = default_cap(*s);
-  if (cap / kTileRows > 65535 || s->E * cap >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
-  if (s->T * s->topk >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  const int64_t ne = s->E + (shared ? 1 : 0), nk = s->topk + (shared ? 1 : 0);
+  if (cap / kTileRows > 65535 || ne * cap >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (s->T * nk >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
   if (s->identity_experts) return MOE_OK;
   if (s->I <= 0 || s->I > (1 << 24) || s->I % 16 != 0) return MOE_ERR_INVALID_ARG;
   if (!is_dtype(s->weight_dtype) || !is_dtype(s->h_dtype) || !is_dtype(s->y_dtype))
@@ -57,8 +61,11 @@ moe_status make_ctx(const moe_shape* s, void* ws, moe_stream_t stream, Ctx* c) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
   if (!ws || ((uintptr_t)ws & 255u) != 0) return MOE_ERR_INVALID_ARG;
-  c->s = *s;
-  c->L = make_layout(*s);
+  c->s = effective_shape(*s);
+  c->routed_E = s->E;
+  c->routed_k = s->topk;
+  c->shared = (s->flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0;
+  c->L = make_layout(c->s);
   c->ws = ws_view(ws, c->L);
   c->stream = (cudaStream_t)stream;
   int dev = 0;
@@ -150,7 +157,7 @@ moe_status moe_workspace_bytes(const moe_shape* shape, size_t* bytes) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (!bytes) return MOE_ERR_INVALID_ARG;
-  *bytes = make_layout(*shape).total;
+  *bytes = make_layout(effective_shape(*shape)).total;
   return MOE_OK;
 }
 
@@ -204,10 +211,10 @@ moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits,
   if (!tok_ok(c, logits) || !tok_ok(c, topk_idx) || !tok_ok(c, topk_w) || !aligned16(logits) ||
       !tok_ok(c, x) || !aligned16(x) || !tok_ok(c, out) || !aligned16(out))
     return MOE_ERR_INVALID_ARG;
-  st = check_bufs(shape, bufs, true);
+  st = check_bufs(&c.s, bufs, true);
   if (st != MOE_OK) return st;
   if (!shape->identity_experts) {
-    st = check_weights(shape, w);
+    st = check_weights(&c.s, w);
     if (st != MOE_OK) return st;
     if (!y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   }

@@ -201,8 +201,22 @@ moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_
 
 // ---- launchers (host, internal) --------------------------------------------
 
+// The shape the dispatch, grouped FFN and combine kernels work on: a shared
+// expert is expert E of E + 1 and every token's slot k of k + 1 (weight 1).
+inline moe_shape effective_shape(const moe_shape& s) {
+  moe_shape e = s;
+  if (s.flags & MOE_FLAG_SHARED_EXPERT) {
+    e.E += 1;
+    e.topk += 1;
+  }
+  return e;
+}
+
 struct Ctx {
-  moe_shape s;
+  moe_shape s;        // effective shape (see effective_shape)
+  int64_t routed_E;   // logits per token
+  int64_t routed_k;   // experts chosen by the router
+  int shared;         // 1: slot routed_k of every token is the shared expert
   Layout L;
   Ws ws;
   cudaStream_t stream;

@@ -28,7 +28,7 @@ __device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
 
 template <int NV>  // logits per lane (multiple of 4 when VEC)
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-route_kernel(const float* __restrict__ logits, int T, int E, int k, int renorm,
+route_kernel(const float* __restrict__ logits, int T, int E, int k, int renorm, int shared,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, Header* hdr) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -102,9 +102,15 @@ route_kernel(const float* __restrict__ logits, int T, int E, int k, int renorm,
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  // with a shared expert each token's row has k + 1 slots, the last being
+  // the shared expert (index E) with weight 1
+  const int ks = k + shared;
   if (lane < k) {
-    topk_idx[(int64_t)t * k + lane] = sel_i;
-    topk_w[(int64_t)t * k + lane] = expf(sel_v - top) / part;
+    topk_idx[(int64_t)t * ks + lane] = sel_i;
+    topk_w[(int64_t)t * ks + lane] = expf(sel_v - top) / part;
+  } else if (shared && lane == k) {
+    topk_idx[(int64_t)t * ks + k] = E;
+    topk_w[(int64_t)t * ks + k] = 1.f;
   }
 }
 
@@ -114,14 +120,14 @@ cudaError_t go(const Ctx& c, const float* logits, int32_t* idx, float* w) {
   if (T == 0) return cudaSuccess;
   dim3 grid((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   route_kernel<NV><<<grid, kWarpsPerBlock * 32, 0, c.stream>>>(
-      logits, T, (int)c.s.E, (int)c.s.topk, c.s.renorm, idx, w, c.ws.hdr);
+      logits, T, (int)c.routed_E, (int)c.routed_k, c.s.renorm, c.shared, idx, w, c.ws.hdr);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float* w) {
-  const int64_t E = c.s.E;
+  const int64_t E = c.routed_E;
   if (E <= 128) return go<4>(c, logits, idx, w);
   if (E <= 256) return go<8>(c, logits, idx, w);
   if (E <= 512) return go<16>(c, logits, idx, w);

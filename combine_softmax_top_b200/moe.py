@@ -118,7 +118,7 @@ def make_shape(s: Spec, T: int | None = None) -> moe_shape:
     sh.weight_dtype, sh.h_dtype, sh.y_dtype, sh.out_dtype = _DT[s.weight], _DT[s.h], _DT[s.y], _DT[s.out]
     sh.renorm, sh.identity_experts = s.renorm, s.identity
     sh.cap_rows = s.cap_rows
-    sh.quant_block, sh.flags = 128, 0
+    sh.quant_block, sh.flags = 128, (1 if s.shared else 0)   # 1: MOE_FLAG_SHARED_EXPERT
     return sh
 
 
@@ -217,20 +217,21 @@ def alloc_buffers(s: Spec, device="cuda", T: int | None = None, stream=None) -> 
     sh = make_shape(s, T)
     T = sh.T
     cap = s.cap_rows if s.cap_rows else max(128, -(-T // 128) * 128)
-    rows = s.E * cap
+    ne, ks = s.E + s.shared, s.k + s.shared   # a shared expert adds one expert and one slot
+    rows = ne * cap
     nws = moe_workspace_bytes(sh)
     ws = torch.empty(nws, dtype=torch.uint8, device=device)
     z = dict(device=device)
     bufs = Buffers(
         shape=sh, spec=s, ws=ws,
-        topk_idx=torch.empty((T, s.k), dtype=torch.int32, **z),
-        topk_w=torch.empty((T, s.k), dtype=torch.float32, **z),
+        topk_idx=torch.empty((T, ks), dtype=torch.int32, **z),
+        topk_w=torch.empty((T, ks), dtype=torch.float32, **z),
         xq=torch.empty((rows, s.H), dtype=_TORCH[s.xq], **z),
         xs=torch.empty((rows, s.H // 128), dtype=torch.float32, **z) if s.xq == E4M3 else None,
-        counts=torch.empty(s.E, dtype=torch.int32, **z),
-        offsets=torch.empty(s.E, dtype=torch.int32, **z),
+        counts=torch.empty(ne, dtype=torch.int32, **z),
+        offsets=torch.empty(ne, dtype=torch.int32, **z),
         row_src=torch.full((rows,), -1, dtype=torch.int32, **z),
-        pos=torch.empty(T * s.k, dtype=torch.int32, **z),
+        pos=torch.empty(T * ks, dtype=torch.int32, **z),
         hq=None if s.identity else torch.empty((rows, s.I), dtype=_TORCH[s.h], **z),
         hs=torch.empty((rows, s.I // 128), dtype=torch.float32, **z)
         if (not s.identity and s.h == E4M3) else None,

@@ -47,6 +47,7 @@ class Spec:
     w_std: float = 0.02
     zipf_s: float = 0.0   # > 0: add log p_e, p_e proportional to (e+1)^-s, to the logits
     cap_rows: int = 0     # 0: default round_up(T, 128)
+    shared: int = 0       # 1: one shared expert (index E) every token also goes through, weight 1
     extra: dict = field(default_factory=dict)
 
     def with_(self, **kw) -> "Spec":
@@ -55,6 +56,16 @@ class Spec:
     @property
     def cap(self) -> int:
         return self.cap_rows if self.cap_rows else max(128, -(-self.T // 128) * 128)
+
+    @property
+    def ne(self) -> int:
+        """Experts with weights and windows (the shared one included)."""
+        return self.E + self.shared
+
+    @property
+    def ks(self) -> int:
+        """Slots per token (the shared expert's included)."""
+        return self.k + self.shared
 
 
 # The five workloads of the layer (tiny fp32, decode, prefill, skewed routing,
@@ -102,19 +113,20 @@ def _block_quantize_weights(w: torch.Tensor):
 
 def _weights(s: Spec, seed: int, tag: int, rows: int, cols: int, device, chunk: int = 16):
     g = _gen(seed, tag, device)
+    ne = s.ne
     if s.weight == E4M3:
-        q = torch.empty((s.E, rows, cols), dtype=torch.uint8, device=device)
-        sc = torch.empty((s.E, rows // 128, cols // 128), dtype=torch.float32, device=device)
-        for e0 in range(0, s.E, chunk):
-            n = min(chunk, s.E - e0)
+        q = torch.empty((ne, rows, cols), dtype=torch.uint8, device=device)
+        sc = torch.empty((ne, rows // 128, cols // 128), dtype=torch.float32, device=device)
+        for e0 in range(0, ne, chunk):
+            n = min(chunk, ne - e0)
             w = torch.randn((n, rows, cols), generator=g, device=device) * s.w_std
             q[e0:e0 + n], sc[e0:e0 + n] = _block_quantize_weights(w)
             del w
         return q, sc
-    out = torch.empty((s.E, rows, cols), dtype=torch.float32 if s.weight == F32 else torch.bfloat16,
+    out = torch.empty((ne, rows, cols), dtype=torch.float32 if s.weight == F32 else torch.bfloat16,
                       device=device)
-    for e0 in range(0, s.E, chunk):
-        n = min(chunk, s.E - e0)
+    for e0 in range(0, ne, chunk):
+        n = min(chunk, ne - e0)
         w = torch.randn((n, rows, cols), generator=g, device=device) * s.w_std
         out[e0:e0 + n] = w.to(out.dtype)
     return out, None
@@ -122,7 +134,8 @@ def _weights(s: Spec, seed: int, tag: int, rows: int, cols: int, device, chunk: 
 
 def make_inputs(s: Spec, seed: int = 0, device="cpu", with_weights: bool = True) -> dict:
     """Router logits [T, E] fp32, activations x [T, H], and (unless identity
-    experts) W_gate/W_up [E, I, H], W_down [E, H, I] with e4m3 block scales."""
+    experts) W_gate/W_up [E', I, H], W_down [E', H, I] with e4m3 block scales,
+    E' = E + shared (the shared expert last)."""
     dev = torch.device(device)
     logits = torch.randn((s.T, s.E), generator=_gen(seed, 0, dev), device=dev)
     if s.zipf_s > 0:

@@ -87,7 +87,21 @@ typedef enum moe_status {
  * cap_rows, when given, must be a multiple of 128.
  * Routing weights are the softmax over all E logits of the selected experts,
  * renormalised over the k selected ones when renorm = 1.
+ *
+ * flags = MOE_FLAG_SHARED_EXPERT adds one shared expert that every token also
+ * goes through, computed in the same grouped FFN launch and added to the
+ * output with weight 1 (GC-MoE feed item: the compute partition fuses
+ * "optionally shared experts"; the weight-1 sum is this library's reading).
+ * E and topk stay the routed counts (logits are [T, E]); every per-expert and
+ * per-pair array grows by one: the weight arrays hold E + 1 experts (the
+ * shared one last, index E), topk_idx / topk_w have topk + 1 columns (moe_route
+ * writes E and 1.0 into the last), the windows hold E + 1 experts
+ * (counts / offsets [E + 1], rows (E + 1) * cap) and pos has T * (topk + 1)
+ * entries. cap must cover all T tokens; topk + 1 <= 32; not with identity
+ * experts.
  */
+enum { MOE_FLAG_SHARED_EXPERT = 1 };
+
 typedef struct moe_shape {
   int64_t T;              /* tokens, >= 0 */
   int64_t H;              /* hidden size */
@@ -104,7 +118,7 @@ typedef struct moe_shape {
   int32_t identity_experts; /* 1: every expert returns its input (no FFN) */
   int64_t cap_rows;       /* rows per expert window; 0 = round_up(T, 128) */
   int32_t quant_block;    /* must be 128 */
-  int32_t flags;          /* reserved, must be 0 */
+  int32_t flags;          /* 0, or MOE_FLAG_SHARED_EXPERT */
 } moe_shape;
 
 /*

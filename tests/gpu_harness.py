@@ -38,9 +38,10 @@ def oracle_problem(s: W.Spec, inp: dict, experts=None) -> oracle.Problem:
     """Oracle problem for `s`; weights of only `experts` (all if None) are
     copied to the host."""
     kw = dict(x_dtype=ODT[s.act], xq_dtype=ODT[s.xq], w_dtype=ODT[s.weight], h_dtype=ODT[s.h],
-              y_dtype=ODT[s.y], out_dtype=ODT[s.out], renorm=s.renorm, identity=s.identity)
+              y_dtype=ODT[s.y], out_dtype=ODT[s.out], renorm=s.renorm, identity=s.identity,
+              shared=s.shared)
     if not s.identity:
-        es = range(s.E) if experts is None else sorted(set(int(e) for e in experts))
+        es = range(s.ne) if experts is None else sorted(set(int(e) for e in experts) | ({s.E} if s.shared else set()))
         for name in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
             t = inp.get(name)
             if t is not None:
@@ -51,10 +52,10 @@ def oracle_problem(s: W.Spec, inp: dict, experts=None) -> oracle.Problem:
 def placed_rows(b: moe.Buffers):
     """(row ids, pair ids, expert ids) of every filled row, from counts/row_src."""
     counts = b.counts.cpu().numpy()
-    cap = b.xq.shape[0] // b.spec.E
+    cap = b.xq.shape[0] // b.spec.ne
     rows = np.concatenate([e * cap + np.arange(c) for e, c in enumerate(counts)]) if counts.sum() \
         else np.zeros(0, np.int64)
-    experts = np.repeat(np.arange(b.spec.E), counts)
+    experts = np.repeat(np.arange(b.spec.ne), counts)
     pairs = b.row_src.cpu().numpy()[rows]
     return rows.astype(np.int64), pairs.astype(np.int64), experts.astype(np.int32)
 

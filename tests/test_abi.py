@@ -49,7 +49,7 @@ def test_workspace_grows_with_capacity():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("topk", 0), ("topk", 33), ("E", 0), ("H", 100), ("quant_block", 64), ("flags", 1),
+    ("topk", 0), ("topk", 33), ("E", 0), ("H", 100), ("quant_block", 64), ("flags", 2),
     ("cap_rows", 100), ("renorm", 2), ("T", -1), ("act_dtype", 7),
 ])
 def test_invalid_shapes_rejected_on_host(field, value):
@@ -59,6 +59,30 @@ def test_invalid_shapes_rejected_on_host(field, value):
     assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 1
     # every entry point checks the shape first, before any CUDA call
     assert moe.lib().moe_route(ctypes.byref(sh), None, None, None, None, None) == 1
+
+
+@pytest.mark.parametrize("base,over", [
+    ("sweep", {}),                          # identity experts have no FFN to share
+    ("decode", {"topk": 32}),               # topk + 1 slots > 32
+    ("decode", {"cap_rows": 0, "T": 200}),  # placeholder: cap set below T
+])
+def test_shared_expert_preconditions(base, over):
+    """The shared expert takes every token (cap >= T), one more slot per token
+    (topk + 1 <= 32), and needs real experts."""
+    sh = moe.make_shape(W.spec(base, shared=1))
+    for f, v in over.items():
+        setattr(sh, f, v)
+    if "T" in over:
+        sh.cap_rows = 128                   # 128 < T = 200
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 1
+
+
+def test_shared_expert_workspace_covers_one_more_expert():
+    s = W.spec("decode")
+    a = moe.moe_workspace_bytes(moe.make_shape(s))
+    b = moe.moe_workspace_bytes(moe.make_shape(s.with_(shared=1)))
+    assert b > a
 
 
 def test_unsupported_dtype_combination():
