@@ -45,27 +45,36 @@ constexpr int kSlab = 128;      // K bytes per slab (one 128-byte swizzle row)
 constexpr int kABytes = 128 * kSlab;   // 128 weight rows of one slab
 constexpr int kMaxDynSmem = 232448;    // 227 KB per CTA
 constexpr int kCtlBytes = 2048;        // barriers, job queue, flags, reductions
-constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert first-tile table (E <= 1024)
+constexpr int kTileTabBytes = 4 * 1025 + 252;   // per-expert chunk table (E <= 1024)
+// With 128-row tiles, an expert's last tile of at most kTailMax rows joins
+// the tile before it: one job of up to 128 + kTailMax rows.
+constexpr int kTailMax = 32;
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
-// A0 | A1 | B (kBRows x 128 B, or two slabs of N rows) | SFA0 | SFA1 | SFB0
+// A0 | A1 | B (kBRows (+ kTailMax) x 128 B, or two slabs of N rows) | SFA0 |
+// SFA1 | SFB0 | SFB1 (the joined tail's token scales)
 template <int kBRows>
 struct Stage {
+  static constexpr int kBRowsMax = kBRows + (kBRows > 64 ? kTailMax : 0);
   static constexpr int kOffA1 = kABytes;
   static constexpr int kOffB = 2 * kABytes;
-  static constexpr int kOffSfa0 = kOffB + kBRows * kSlab;
+  static constexpr int kOffSfa0 = kOffB + kBRowsMax * kSlab;
   static constexpr int kOffSfa1 = kOffSfa0 + kSfAtomBytes;
   static constexpr int kOffSfb0 = kOffSfa1 + kSfAtomBytes;
-  static constexpr int kStride = (kOffSfb0 + kSfAtomBytes + 1023) / 1024 * 1024;
+  static constexpr int kOffSfb1 = kOffSfb0 + kSfAtomBytes;
+  static constexpr int kStride = (kOffSfb1 + kSfAtomBytes + 1023) / 1024 * 1024;
   static constexpr int kStages = (kMaxDynSmem - kCtlBytes - kTileTabBytes - 1024) / kStride;
   static constexpr int kBarOffset = kStages * kStride;
   static constexpr int kSmemBytes = kBarOffset + kCtlBytes + kTileTabBytes + 1024 /* alignment slack */;
   static_assert(kStages >= 3, "pipeline depth");
+  static_assert(kBRows <= 64 || kStages >= 4, "the joined tail keeps four stages");
 };
 
 constexpr uint32_t kTmemCols = 512;
-// accumulators: two 128-column slots at columns 0 and 128; scale factors after
-constexpr uint32_t kColSfa0 = 256, kColSfa1 = 260, kColSfb0 = 264;
+// accumulators: two 128-column slots at columns 0 and 128 (a job with a joined
+// tail: gate at 0, up at N, N <= 128 + kTailMax); scale factors from column
+// 448, the tokens' over 8 columns (256 rows)
+constexpr uint32_t kColSfa0 = 448, kColSfa1 = 452, kColSfb0 = 456;
 
 enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
 // counter-set misc slots used here: FFN calls completed on this dispatch, CTAs
@@ -95,11 +104,13 @@ struct TcParams {
 struct Job {
   int e, tile, slice, rows, row_off, kind, nslab, slot;
   int pair;   // down job over two 128-feature slices of H (slice, slice + 1)
+  int wide;   // tile `tile` with the expert's short last tile joined (rows > 128)
 };
 
 __device__ __forceinline__ int4 pack_job(const Job& j) {
   return make_int4(j.e, j.tile | (j.slice << 16),
-                   j.rows | (j.row_off << 8) | (j.kind << 16) | (j.nslab << 20) | (j.pair << 24), j.slot);
+                   j.rows | (j.row_off << 8) | (j.kind << 16) | (j.nslab << 20) | (j.pair << 24) | (j.wide << 25),
+                   j.slot);
 }
 
 __device__ __forceinline__ Job unpack_job(int4 v) {
@@ -112,6 +123,7 @@ __device__ __forceinline__ Job unpack_job(int4 v) {
   j.kind = (v.z >> 16) & 0xF;
   j.nslab = (v.z >> 20) & 0xF;
   j.pair = (v.z >> 24) & 0x1;
+  j.wide = (v.z >> 25) & 0x1;
   j.slot = v.w;
   return j;
 }
@@ -247,8 +259,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   // down units cover two slices of H each when tiles are large (the two share
   // the token tile, like gate and up)
   const int dpair = (kBRows > 64 && (p.n_hslices & 1) == 0) ? 2 : 1;
-  const uint32_t n1 = ntiles * (uint32_t)p.n_islices;
-  const uint32_t total = n1 + ntiles * (uint32_t)(p.n_hslices / dpair);
   Header* hdr = p.ws.hdr;
 
   // Take job i from the queue (one lane of a consumer role).
@@ -269,30 +279,51 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // of one expert with the same weight slice and share it in L2.
     // For each unit the scheduler waits for the tile's sentinel (and a down
     // unit's h), splits the tile into chunks of <= kBRows rows and queues them.
-    int* tile_pre = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1] first tile of each expert
+    // Per expert, its first chunk (low 24 bits) and the rows of a joined tail
+    // (high 8 bits). A chunk is one tile, except that with 128-row tiles an
+    // expert's last tile of at most kTailMax rows joins the tile before it:
+    // its weights are then not streamed again for a few tokens.
+    int* chunk_tab = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1]
+    int ntab = 0;   // tiles counted from the expert counts (lane 31)
     {
       const uint32_t* cnt = set_count(set);
       const int per = (p.E + 31) / 32;
-      int local = 0;
-      for (int i = 0; i < per; ++i) {
-        const int e = lane * per + i;
-        if (e < p.E) local += ((int)min(ld_acquire(cnt + e), (uint32_t)p.cap) + kTileRows - 1) / kTileRows;
-      }
-      int incl = local;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      int run = incl - local;
+      auto tiles_of = [&](int e, int* tail) {
+        const int c = (int)min(ld_acquire(cnt + e), (uint32_t)p.cap);
+        const int nt = (c + kTileRows - 1) / kTileRows;
+        const int last = c - (nt - 1) * kTileRows;
+        *tail = (kBRows > 64 && nt >= 2 && last <= kTailMax) ? last : 0;
+        return nt;
+      };
+      int lt = 0, lc = 0;
       for (int i = 0; i < per; ++i) {
         const int e = lane * per + i;
         if (e < p.E) {
-          tile_pre[e] = run;
-          run += ((int)min(ld_acquire(cnt + e), (uint32_t)p.cap) + kTileRows - 1) / kTileRows;
+          int tail;
+          const int nt = tiles_of(e, &tail);
+          lt += nt;
+          lc += nt - (tail ? 1 : 0);
         }
       }
-      if (lane == 31) tile_pre[p.E] = incl;
+      int it = lt, ic = lc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int vt = __shfl_up_sync(0xffffffffu, it, off);
+        const int vc = __shfl_up_sync(0xffffffffu, ic, off);
+        if (lane >= off) { it += vt; ic += vc; }
+      }
+      int rc = ic - lc;
+      for (int i = 0; i < per; ++i) {
+        const int e = lane * per + i;
+        if (e < p.E) {
+          int tail;
+          const int nt = tiles_of(e, &tail);
+          chunk_tab[e] = rc | (tail << 24);
+          rc += nt - (tail ? 1 : 0);
+        }
+      }
+      if (lane == 31) chunk_tab[p.E] = ic;
+      ntab = __shfl_sync(0xffffffffu, it, 31);
       __syncwarp();
     }
     if (lane == 0) {
@@ -306,12 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         ++i;
         return true;
       };
-      const uint32_t ntab = (uint32_t)tile_pre[p.E];
-      if (ntab != ntiles) {   // the published tile total disagrees with the counts
-        latch_error(hdr, MOE_ERR_INVALID_ARG, 0x24000000u | ntab);
+      if ((uint32_t)ntab != ntiles) {   // the published tile total disagrees with the counts
+        latch_error(hdr, MOE_ERR_INVALID_ARG, 0x24000000u | (uint32_t)ntab);
         *abort_flag = 1;
         good = false;
       }
+      const uint32_t nchunks = (uint32_t)(chunk_tab[p.E] & 0xFFFFFF);
+      const uint32_t n1 = nchunks * (uint32_t)p.n_islices;                       // gate/up units
+      const uint32_t total = n1 + nchunks * (uint32_t)(p.n_hslices / dpair);   // + down units
       // units are taken from one counter in increasing order (dynamic load
       // balance); every unit waits only on units earlier in that order
       while (good) {
@@ -321,37 +354,45 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         j.kind = u >= n1 ? kKindDown : kKindGateUp;
         const uint32_t v = j.kind == kKindDown ? u - n1 : u;
         const uint32_t ns = (uint32_t)(j.kind == kKindDown ? p.n_hslices / dpair : p.n_islices);
-        // expert: the last e with tile_pre[e] * ns <= v (empty experts never are)
+        // expert: the last e with first_chunk[e] * ns <= v (empty experts never are)
         int lo = 0, hi = p.E - 1;
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
-          if ((uint32_t)tile_pre[mid] * ns <= v) lo = mid;
+          if ((uint32_t)(chunk_tab[mid] & 0xFFFFFF) * ns <= v) lo = mid;
           else hi = mid - 1;
         }
         j.e = lo;
-        const uint32_t nt = (uint32_t)(tile_pre[lo + 1] - tile_pre[lo]);
-        const uint32_t w = v - (uint32_t)tile_pre[lo] * ns;
+        const int c0 = chunk_tab[lo] & 0xFFFFFF;
+        const int tail = (int)((uint32_t)chunk_tab[lo] >> 24);
+        const uint32_t nc = (uint32_t)((chunk_tab[lo + 1] & 0xFFFFFF) - c0);
+        const uint32_t w = v - (uint32_t)c0 * ns;
         j.pair = j.kind == kKindDown && dpair == 2;
-        j.slice = (int)(w / nt) * (j.pair ? 2 : 1);
-        j.tile = (int)(w % nt);
+        j.slice = (int)(w / nc) * (j.pair ? 2 : 1);
+        j.tile = (int)(w % nc);
         j.slot = j.e * p.tpe + j.tile;     // global tile id: the down units' counter
+        j.wide = tail && j.tile == (int)nc - 1;
         int rows = 0;
         good = wait_tile(p, epoch, j.e, j.tile, abort_flag, &rows);
+        if (good && j.wide) {   // the joined tail's sentinel too
+          int rows2 = 0;
+          good = wait_tile(p, epoch, j.e, j.tile + 1, abort_flag, &rows2);
+          rows += rows2;
+        }
         if (!good) break;
-        const int nch = (rows + kBRows - 1) / kBRows;
+        const int nch = j.wide ? 1 : (rows + kBRows - 1) / kBRows;
         if (j.kind == kKindDown)
           good = wait_count(hdone + j.slot, (uint32_t)(p.n_islices * nch) * (gen + 1u), abort_flag, hdr,
                             0x30000000u | (uint32_t)j.slot);
         for (int c = 0; good && c < nch; ++c) {
           j.row_off = c * kBRows;
-          j.rows = min(kBRows, rows - j.row_off);
+          j.rows = j.wide ? rows : min(kBRows, rows - j.row_off);
           const int N = (j.rows + 15) & ~15;
           j.nslab = (j.kind == kKindDown && !j.pair && 2 * N <= kBRows && (p.nk2 & 1) == 0) ? 2 : 1;
           good = push(j);
         }
       }
       Job end;
-      end.e = end.tile = end.slice = end.rows = end.row_off = end.slot = end.pair = 0;
+      end.e = end.tile = end.slice = end.rows = end.row_off = end.slot = end.pair = end.wide = 0;
       end.nslab = 1;
       end.kind = good ? kKindEnd : kKindAbort;
       push(end);   // bounded; consumers also stop on the abort flag
@@ -457,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         // chosen at run time costs about four times as much to issue.
         if (ptx::elect_one()) {
           uint64_t* fb = full + stage;
-          ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (uint32_t)kSfAtomBytes : 0u));
+          ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (j.wide ? 2u : 1u) * (uint32_t)kSfAtomBytes : 0u));
           const int kx0 = kb0 * p.kelems;
           if (down) {
             if constexpr (kBRows <= 64) {
@@ -496,20 +537,25 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               else ptx::tma_load_2d(dst, &p.tm_x[3], fb, kx, brow);
             } else if (down) {
               int r = 0;
+              if (N - r >= 128) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[3], fb, kx, brow + r); r += 128; }
               if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[2], fb, kx, brow + r); r += 64; }
               if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[1], fb, kx, brow + r); r += 32; }
               if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_h[0], fb, kx, brow + r); r += 16; }
             } else {
               int r = 0;
+              if (N - r >= 128) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[3], fb, kx, brow + r); r += 128; }
               if (N - r >= 64) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[2], fb, kx, brow + r); r += 64; }
               if (N - r >= 32) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[1], fb, kx, brow + r); r += 32; }
               if (N - r >= 16) { ptx::tma_load_2d(dst + r * kSlab, &p.tm_x[0], fb, kx, brow + r); r += 16; }
             }
           }
-          if (sf_stage) {   // the tokens' scale atom of this group of four blocks
-            const uint8_t* sf = down ? p.ws.hsf + (tile_g * p.igroups + kb0 / 4) * kSfAtomBytes
-                                     : p.ws.xsf + (tile_g * p.hgroups + kb0 / 4) * kSfAtomBytes;
-            ptx::bulk_load(st + S::kOffSfb0, sf, kSfAtomBytes, fb);
+          if (sf_stage) {   // the tokens' scale atom(s) of this group of four blocks
+            const uint8_t* sfb = down ? p.ws.hsf : p.ws.xsf;
+            const int groups = down ? p.igroups : p.hgroups;
+            ptx::bulk_load(st + S::kOffSfb0, sfb + (tile_g * groups + kb0 / 4) * kSfAtomBytes, kSfAtomBytes, fb);
+            if (j.wide)   // the joined tail tile's atom
+              ptx::bulk_load(st + S::kOffSfb1, sfb + ((tile_g + 1) * groups + kb0 / 4) * kSfAtomBytes, kSfAtomBytes,
+                             fb);
           }
         }
         __syncwarp();
@@ -534,7 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // ---------------------------------------------------------------- MMA issuer
     // Two 128-column accumulator slots: a job with N <= 64 (or a down job)
     // takes one (gate at +0, up at +64), a gate/up job with N > 64 takes both,
-    // so the next job's MMAs overlap the previous job's epilogue.
+    // so the next job's MMAs overlap the previous job's epilogue. A job with
+    // a joined tail (N <= 128 + kTailMax) takes both slots and the columns
+    // after them: gate (or the down slice) at column 0, up (or the second
+    // slice) at N.
     // The whole warp walks the loop with warp-uniform values (descriptors,
     // tensor-memory addresses); lane 0 polls the barriers and one elected
     // lane issues the copies, MMAs and commits.
@@ -550,10 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const bool down = j.kind == kKindDown;
       const bool dual = !down || j.pair;   // two accumulators: gate/up or two slices of H
       const int N = (j.rows + 15) & ~15;
-      const bool two = dual && N > 64;
+      const bool two = j.wide || (dual && N > 64);
       const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
-      const uint32_t colG = 128u * s0;
-      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+      const uint32_t colG = j.wide ? 0u : 128u * s0;
+      const uint32_t colU = j.wide ? (uint32_t)N : (two ? 128u * s1 : 128u * s0 + 64u);
       int ok = 1;
       if (lane == 0) {
         ok = wait_bar(acc_empty + s0, ((acc_ph >> s0) & 1u) ^ 1u, abort_flag, hdr, 0x50000000u | s0);
@@ -585,6 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
               ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
               ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
+              if (j.wide)   // the joined tail's rows 128.. read columns kColSfb0 + 4 ..
+                ptx::tmem_cp_32x128b_x4(tmem + kColSfb0 + 4, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb1), 16, 128, ptx::kLayoutNone));
               if (dual)
                 ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
             }
@@ -670,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         if (!good) jj.kind = kKindAbort;
         if (jj.kind < kKindEnd) {
           const int N = (jj.rows + 15) & ~15;
-          const bool two = (jj.kind == kKindGateUp || jj.pair) && N > 64;
+          const bool two = jj.wide || ((jj.kind == kKindGateUp || jj.pair) && N > 64);
           const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
           good = wait_bar(acc_full + s0, (acc_ph >> s0) & 1u, abort_flag, hdr, 0x70000000u | s0);
           if (good && two) good = wait_bar(acc_full + s1, (acc_ph >> s1) & 1u, abort_flag, hdr, 0x70000000u | s1);
@@ -685,10 +736,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const bool down = j.kind == kKindDown;
       const bool dual = !down || j.pair;
       const int N = (j.rows + 15) & ~15;
-      const bool two = dual && N > 64;
+      const bool two = j.wide || (dual && N > 64);
       const uint32_t s0 = next_slot, s1 = next_slot ^ 1u;
-      const uint32_t colG = 128u * s0;
-      const uint32_t colU = two ? 128u * s1 : 128u * s0 + 64u;
+      const uint32_t colG = j.wide ? 0u : 128u * s0;
+      const uint32_t colU = j.wide ? (uint32_t)N : (two ? 128u * s1 : 128u * s0 + 64u);
       while (!ptx::mbar_try_wait(acc_full + s0, (acc_ph >> s0) & 1u)) {}   // completed: returns at once
       if (two) while (!ptx::mbar_try_wait(acc_full + s1, (acc_ph >> s1) & 1u)) {}
       ptx::tc_fence_after();
@@ -722,18 +773,23 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
           }
         }
       };
-      if (nA > 0) drain(32 * set, vA);
-      if (nB > 0) drain(32 * set + 64, vB);
       // accumulators consumed: let the MMA warp reuse the slot(s)
-      ptx::tc_fence_before();
-      ptx::named_barrier(1, kEpiThreads);
-      if (et == 0) {
-        ptx::mbar_arrive(acc_empty + s0);
-        if (two) ptx::mbar_arrive(acc_empty + s1);
+      auto release = [&]() {
+        ptx::tc_fence_before();
+        ptx::named_barrier(1, kEpiThreads);
+        if (et == 0) {
+          ptx::mbar_arrive(acc_empty + s0);
+          if (two) ptx::mbar_arrive(acc_empty + s1);
+        }
+        acc_ph ^= 1u << s0;
+        if (two) acc_ph ^= 1u << s1;
+        else next_slot ^= 1u;
+      };
+      if (!j.wide) {
+        if (nA > 0) drain(32 * set, vA);
+        if (nB > 0) drain(32 * set + 64, vB);
+        release();
       }
-      acc_ph ^= 1u << s0;
-      if (two) acc_ph ^= 1u << s1;
-      else next_slot ^= 1u;
       // the per-token work on one drained batch: y stores, or the per-token
       // max over the 128 features (one redux per token per warp, the max over
       // the set's four warps and the scale once per token through shared
@@ -766,8 +822,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             if (lane < nv) {
               const int64_t r = row0 + n0 + lane;
               p.hs[r * (p.I / 128) + j.slice] = exp2i(pe);
-              // byte of this slice in the tile's scale atom (row j.row_off + n0 + lane)
-              *sf_atom_byte(p.ws.hsf, tile_g, p.igroups, j.slice, j.row_off + n0 + lane) = (uint8_t)(pe + 127);
+              // byte of this slice in its tile's scale atom (a joined tail's
+              // rows past 128 belong to the next tile)
+              const int rr = j.row_off + n0 + lane;
+              *sf_atom_byte(p.ws.hsf, tile_g + rr / kTileRows, p.igroups, j.slice, rr % kTileRows) = (uint8_t)(pe + 127);
             }
           }
           ptx::named_barrier(set_bar, 128);
@@ -791,8 +849,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
             if (jj < nv) hp[(int64_t)jj * p.I] = __float2bfloat16_rn(__uint_as_float(v[jj]));
         }
       };
-      if (nA > 0) finish(32 * set, nA, vA);
-      if (nB > 0) finish(32 * set + 64, nB, vB);
+      if (!j.wide) {
+        if (nA > 0) finish(32 * set, nA, vA);
+        if (nB > 0) finish(32 * set + 64, nB, vB);
+      } else {   // a joined tail: up to 5 batches, drained and finished one at a time
+        for (int n0 = 32 * set; n0 < j.rows; n0 += 64) {
+          drain(n0, vA);
+          finish(n0, min(32, j.rows - n0), vA);
+        }
+        release();
+      }
       if (!down) {
         // publish this chunk of this slice of h to the down jobs of the tile
         __threadfence();
