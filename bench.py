@@ -39,6 +39,8 @@ def parse():
     p.add_argument("--E", type=int, default=None, help="override the expert count (small profiling cases)")
     p.add_argument("--shared-expert", action="store_true",
                    help="add one shared expert every token also goes through (weight 1)")
+    p.add_argument("--compact", action="store_true",
+                   help="compact expert windows: a counting pass, then windows packed back to back")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -60,6 +62,8 @@ def overrides(args) -> dict:
         o["E"] = args.E
     if getattr(args, "shared_expert", False):
         o["shared"] = 1
+    if getattr(args, "compact", False):
+        o["compact"] = 1
     return o
 
 
@@ -424,7 +428,8 @@ def run_report(args):
     peaks, kind = load_peaks()
     hbm = peaks["hbm_gbs"]
     cases = [W.spec("tiny"), W.spec("decode"), W.spec("prefill"), W.spec("skew"),
-             W.spec("decode", shared=1), W.spec("prefill", shared=1)] + \
+             W.spec("decode", shared=1), W.spec("prefill", shared=1),
+             W.spec("prefill", compact=1), W.spec("skew", compact=1)] + \
         [W.spec("sweep", T=t) for t in W.SWEEP_T]
     for spec in cases:
         inp = W.make_inputs(spec, seed=args.seed, device=dev)
@@ -435,8 +440,10 @@ def run_report(args):
         clk = clocks.stop()
         counts = b.counts.cpu().numpy()
         layer_ms = float(st.sum())
-        line = {"report": spec.name + ("+shared" if spec.shared else ""), "T": spec.T, "H": spec.H, "E": spec.E,
-                "topk": spec.k, "shared_experts": spec.shared,
+        line = {"report": spec.name + ("+shared" if spec.shared else "") + ("+compact" if spec.compact else ""),
+                "T": spec.T, "H": spec.H, "E": spec.E,
+                "topk": spec.k, "shared_experts": spec.shared, "compact_windows": spec.compact,
+                "expert_buffer_rows": spec.rows(),
                 "I": None if spec.identity else spec.I, "dtype": spec.weight if not spec.identity else spec.xq,
                 "layer_us": layer_ms * 1e3, "tokens_per_s": spec.T / (layer_ms / 1e3),
                 "stage_us": {k: float(v * 1e3) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], st)},
@@ -631,6 +638,7 @@ def run_ours(args):
                                    f"top-{spec.k}{' + 1 shared expert' if spec.shared else ''} I={spec.I} "
                                    f"{'e4m3 128x128-block weights, bf16 tokens' if spec.weight == 'e4m3' else spec.weight}",
                        "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I, "shared_experts": spec.shared,
+                       "compact_windows": spec.compact,
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) before every timed step; weights 11 GB > L2"},
             "stage_us": {k: float(stage[:, j].mean() * 1000.0)

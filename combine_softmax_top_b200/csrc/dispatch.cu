@@ -10,9 +10,10 @@
 // abstract).
 //
 // CTAs walk tokens; for each token:
-//  1. lanes j < k claim row e*cap + atomicAdd(count[e], 1) for slot j (the
+//  1. lanes j < k claim row first(e) + atomicAdd(count[e], 1) for slot j (the
 //     expert index loaded two tokens ahead, the atomic issued one token
-//     ahead, so neither round trip stalls the CTA);
+//     ahead, so neither round trip stalls the CTA); first(e) = e * cap, or with
+//     compact windows 128 * base[e] from the counting pass (plan_kernel);
 //  2. all warps stream the token row once (16-byte loads) and write it to the
 //     k claimed rows; E4M3 rows are quantised per 128 values with the
 //     smallest power-of-two scale that keeps the block within +-448, and the
@@ -25,6 +26,12 @@
 //     advances the epoch.
 // Every CTA first zeroes its share of the counter set the *next* dispatch will
 // use, so no separate clean pass is needed.
+//
+// Compact windows (the NVLinkOneSided abstract's Fence protocol: the
+// counts are settled before any row moves, here by stream order between two
+// launches): plan_kernel histograms the expert indices and its last CTA
+// lays the windows out back to back, each rounded up to whole 128-row tiles,
+// so the buffers need T * k + 127 * E rows instead of E * cap.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -37,6 +44,8 @@ struct Args {
   const void* x;
   const int32_t* idx;
   int T, H, E, k, cap, tpe;
+  int compact;         // windows at 128 * base[e] (set_base), sized by the counting pass
+  int64_t tiles;
   int act, xq_dtype;
   moe_dispatch_bufs b;
   Ws ws;
@@ -103,12 +112,13 @@ __device__ __forceinline__ void load16(const void* x, int act, int64_t off, floa
   }
 }
 
-__device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e, int tile,
+// Global tile g (rows 128 g ...) of expert e holds `rows` rows: set its
+// sentinel and append it to the ring.
+__device__ void publish_tile(const Args& a, uint32_t* set, uint32_t epoch, int e, int64_t g,
                              int rows) {
-  st_release(a.ws.sentinel + (int64_t)e * a.tpe + tile, (epoch << 8) | (uint32_t)rows);
+  st_release(a.ws.sentinel + g, (epoch << 8) | (uint32_t)rows);
   const uint32_t slot = atomicAdd(set_misc(set) + kRingHead, 1u);
-  st_release64(a.ws.ring + slot,
-               ((unsigned long long)epoch << 32) | ((unsigned long long)e << 16) | (unsigned)tile);
+  st_release64(a.ws.ring + slot, ring_entry(epoch, e, g));
 }
 
 // Row claims are pipelined over three tokens by the threads tid < k (slot
@@ -124,14 +134,24 @@ __device__ __forceinline__ uint32_t issue_claim(const Args& a, int t, int e, uin
 }
 
 // Token t's slot tid: the claimed row (or -1), recorded in pos/row_src/s_row.
-__device__ __forceinline__ void finish_claim(const Args& a, int t, int tid, int e, uint32_t p, int* s_row, int* s_e) {
+// base: compact windows' first tiles (NULL: windows of cap rows).
+__device__ __forceinline__ void finish_claim(const Args& a, const uint32_t* base, int t, int tid, int e,
+                                             uint32_t p, int* s_row, int* s_e) {
   const int pair = t * a.k + tid;
   int row = -1;
   if (e >= 0 && e < a.E) {
-    if (p < (uint32_t)a.cap) {
-      row = e * a.cap + (int)p;
-      a.b.row_src[row] = pair;
+    uint32_t first, room;
+    if (base) {
+      first = base[e] * (uint32_t)kTileRows;
+      room = base[e + 1] * (uint32_t)kTileRows - first;
     } else {
+      first = (uint32_t)e * (uint32_t)a.cap;
+      room = (uint32_t)a.cap;
+    }
+    if (p < room) {
+      row = (int)(first + p);
+      a.b.row_src[row] = pair;
+    } else {   // compact windows: only if idx changed after the counting pass
       latch_error(a.ws.hdr, MOE_ERR_CAPACITY, (uint32_t)e);
     }
   } else {
@@ -178,7 +198,7 @@ __device__ __forceinline__ void put_slice(const Args& a, int tid, const int* s_r
         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.b.xq) + (int64_t)row * a.H + h0) = qv;
         if (leader) {
           a.b.xs[(int64_t)row * (a.H / kQBlock) + blk] = exp2i(p);
-          if (a.xsf)   // tile id e * tpe + local = row / 128 since cap % 128 == 0
+          if (a.xsf)   // global tile row / 128
             *sf_atom_byte(a.xsf, row / kTileRows, (a.H + 4 * kQBlock - 1) / (4 * kQBlock), blk,
                           row % kTileRows) = (uint8_t)(p + 127);
         }
@@ -251,6 +271,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
   uint32_t* count = set_count(set);
   uint32_t* fill = set_fill(set, a.E);
   uint32_t* misc = set_misc(set);
+  const uint32_t* base = a.compact ? set_base(set, a.E, a.tiles) : nullptr;
 
   // zero this CTA's share of the next counter set
   {
@@ -276,7 +297,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     e1 = load_expert(a, t + G, tid);
     p1 = issue_claim(a, t + G, e1, count);
     e2 = load_expert(a, t + 2 * G, tid);
-    finish_claim(a, t, tid, e0, p0, s_row[0], s_e[0]);
+    finish_claim(a, base, t, tid, e0, p0, s_row[0], s_e[0]);
   }
   if (t < a.T) {
 #pragma unroll
@@ -287,7 +308,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
   for (; t < a.T; t += G) {
     const int tn = t + G;
     if (tid < a.k && tn < a.T) {
-      finish_claim(a, tn, tid, e1, p1, s_row[cur ^ 1], s_e[cur ^ 1]);   // claimed a token ago
+      finish_claim(a, base, tn, tid, e1, p1, s_row[cur ^ 1], s_e[cur ^ 1]);   // claimed a token ago
       p1 = issue_claim(a, tn + G, e2, count);
       e1 = e2;
       e2 = load_expert(a, tn + 2 * G, tid);
@@ -305,11 +326,9 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     if (tid < a.k) {
       const int row = s_row[cur][tid];
       if (row >= 0) {
-        const int e = s_e[cur][tid];
-        const int local = row - e * a.cap;
-        const int tile = local / kTileRows;
-        const uint32_t old = atomicAdd(fill + (int64_t)e * a.tpe + tile, 1u);
-        if (old + 1 == (uint32_t)kTileRows) publish_tile(a, set, epoch, e, tile, kTileRows);
+        const int g = row / kTileRows;   // windows start on tile boundaries
+        const uint32_t old = atomicAdd(fill + g, 1u);
+        if (old + 1 == (uint32_t)kTileRows) publish_tile(a, set, epoch, s_e[cur][tid], g, kTileRows);
       }
     }
 #pragma unroll
@@ -329,12 +348,13 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
   __syncthreads();
   for (int e = tid; e < a.E; e += kThreads) {
     const uint32_t c_raw = ld_acquire(count + e);
-    const int c = (int)min(c_raw, (uint32_t)a.cap);
+    const int first = base ? (int)base[e] : e * a.tpe;   // global tile
+    const int c = (int)min(c_raw, base ? (base[e + 1] - base[e]) * (uint32_t)kTileRows : (uint32_t)a.cap);
     a.b.counts[e] = c;
-    a.b.offsets[e] = e * a.cap;
+    a.b.offsets[e] = first * kTileRows;
     const int full = c / kTileRows;
     const int rem = c % kTileRows;
-    if (rem) publish_tile(a, set, epoch, e, full, rem);   // the partial last tile
+    if (rem) publish_tile(a, set, epoch, e, first + full, rem);   // the partial last tile
     atomicAdd(&s_tiles, (uint32_t)(full + (rem ? 1 : 0)));
   }
   __threadfence();
@@ -345,6 +365,69 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(Args a) {
     __threadfence();
     a.ws.hdr->epoch_next = epoch + 1;
   }
+}
+
+// ---- compact windows: the counting pass --------------------------------------
+
+constexpr int kPlanThreads = 256;
+
+struct PlanArgs {
+  const int32_t* idx;
+  int64_t pairs;   // T * k
+  int E;
+  int64_t tiles;   // set layout
+  Ws ws;
+};
+
+// Count each expert's (token, slot) pairs into pre[], then (last CTA) lay
+// the windows out: base[e] = sum over e' < e of ceil(pre[e'] / 128),
+// base[E] = the total. Indices outside [0, E) are skipped here; the
+// dispatch kernel reports them.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  extern __shared__ uint32_t hist[];   // [E]
+  __shared__ uint32_t s_last;
+  __shared__ uint32_t s_warp[kPlanThreads / 32];
+  const int tid = threadIdx.x;
+  uint32_t* set = a.ws.set[a.ws.hdr->epoch_next & 1];
+  uint32_t* pre = set_pre(set, a.E, a.tiles);
+  uint32_t* base = set_base(set, a.E, a.tiles);
+  for (int e = tid; e < a.E; e += kPlanThreads) hist[e] = 0u;
+  __syncthreads();
+  for (int64_t i = (int64_t)blockIdx.x * kPlanThreads + tid; i < a.pairs; i += (int64_t)gridDim.x * kPlanThreads) {
+    const int e = __ldg(a.idx + i);
+    if (e >= 0 && e < a.E) atomicAdd(hist + e, 1u);
+  }
+  __syncthreads();
+  for (int e = tid; e < a.E; e += kPlanThreads)
+    if (hist[e]) atomicAdd(pre + e, hist[e]);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(set_misc(set) + kPlanDone, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // exclusive scan of the tile counts: thread tid owns experts
+  // [tid * per, (tid + 1) * per)
+  const int per = (a.E + kPlanThreads - 1) / kPlanThreads;
+  const int e0 = min(a.E, tid * per), e1 = min(a.E, e0 + per);
+  uint32_t own = 0;
+  for (int e = e0; e < e1; ++e) own += (ld_acquire(pre + e) + kTileRows - 1) / kTileRows;
+  uint32_t incl = own;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  uint32_t run = incl - own;
+  for (int w = 0; w < warp; ++w) run += s_warp[w];
+  for (int e = e0; e < e1; ++e) {
+    base[e] = run;
+    run += (ld_acquire(pre + e) + kTileRows - 1) / kTileRows;
+  }
+  if (tid == kPlanThreads - 1) base[a.E] = run;   // the last thread's running total is the sum
 }
 
 }  // namespace
@@ -360,12 +443,27 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
   a.k = (int)c.s.topk;
   a.cap = (int)c.L.cap;
   a.tpe = (int)c.L.tpe;
+  a.compact = c.L.compact ? 1 : 0;
+  a.tiles = c.L.tiles;
   a.act = c.s.act_dtype;
   a.xq_dtype = c.s.xq_dtype;
   a.b = b;
   a.ws = c.ws;
   a.xsf = write_sf && c.s.xq_dtype == MOE_E4M3 ? c.ws.xsf : nullptr;
   a.set_words = (int64_t)c.L.set_words;
+  if (a.compact) {
+    PlanArgs pa;
+    pa.idx = idx;
+    pa.pairs = (int64_t)a.T * a.k;
+    pa.E = a.E;
+    pa.tiles = a.tiles;
+    pa.ws = a.ws;
+    const int64_t want = (pa.pairs + 8 * kPlanThreads - 1) / (8 * kPlanThreads);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, c.num_sms));
+    plan_kernel<<<grid, kPlanThreads, (size_t)a.E * 4, c.stream>>>(pa);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   // one wave of resident CTAs, each walking several tokens (fewer CTAs also
   // means fewer arrivals on the closing counter)
   auto go = [&](auto kern, int& resident) {

@@ -65,6 +65,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x
                                            const moe_dispatch_bufs* bufs, moe_stream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
+  // compact windows need the counting pass's words in a workspace
+  if (shape->flags & MOE_FLAG_COMPACT) return MOE_ERR_UNSUPPORTED;
   if (shape->T > 0 && (!x || !topk_idx)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
   Ctx c;

@@ -22,7 +22,8 @@ struct Args {
   void* y;
   const void* wg;  const void* wu;  const void* wd;
   const float* sg; const float* su; const float* sd;
-  int H, I, E, cap, tpe;
+  int H, I, E;
+  int64_t tiles;                        // global tiles in the expert buffers
   int xq_dt, w_dt, h_dt, y_dt;
   Ws ws;
   uint8_t* hsf;
@@ -34,27 +35,27 @@ __device__ __forceinline__ float ld_act(const void* p, int dt, int64_t i) {
   return e4m3_to_f32(reinterpret_cast<const uint8_t*>(p)[i]);
 }
 
-// Find the tile behind ring slot `slot` for the current epoch (bounded wait).
+// Find the global tile behind ring slot `slot` for the current epoch (bounded wait).
 __device__ bool fetch_tile(const Args& a, uint32_t epoch, uint32_t slot, int* e, int* tile,
                            int* rows) {
   const unsigned long long t0 = globaltimer();
   unsigned long long ent;
   while (true) {
     ent = ld_acquire64(a.ws.ring + slot);
-    if ((uint32_t)(ent >> 32) == epoch) break;
+    if ((uint32_t)(ent >> 40) == (epoch & 0xFFFFFFu)) break;
     if (globaltimer() - t0 > kWaitBudgetNs) {
       latch_error(a.ws.hdr, MOE_ERR_TIMEOUT, slot);
       return false;
     }
     __nanosleep(256);
   }
-  *e = (int)((ent >> 16) & 0xFFFF);
-  *tile = (int)(ent & 0xFFFF);
-  if (*e >= a.E || *tile >= a.tpe) {          // never published: a corrupt workspace
+  *e = (int)((ent >> 24) & 0xFFFF);
+  *tile = (int)(ent & 0xFFFFFF);
+  if (*e >= a.E || *tile >= a.tiles) {          // never published: a corrupt workspace
     latch_error(a.ws.hdr, MOE_ERR_INVALID_ARG, slot);
     return false;
   }
-  const uint32_t* sp = a.ws.sentinel + (int64_t)(*e) * a.tpe + *tile;
+  const uint32_t* sp = a.ws.sentinel + *tile;
   while (true) {
     const uint32_t s = ld_acquire(sp);
     if ((s >> 8) == (epoch & 0xFFFFFFu)) {
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(Args a) {
     const int e = s_info[0], tile = s_info[1], rows = s_info[2];
     __syncthreads();
     if (e < 0) continue;
-    const int64_t row0 = (int64_t)e * a.cap + (int64_t)tile * kTileRows;
+    const int64_t row0 = (int64_t)tile * kTileRows;   // global tile
     const int f0 = slice * kF;
     const void* w0 = DOWN ? a.wd : a.wg;
     const void* w1 = a.wu;
@@ -246,7 +247,7 @@ cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_
   a.wg = w.w_gate; a.wu = w.w_up; a.wd = w.w_down;
   a.sg = w.s_gate; a.su = w.s_up; a.sd = w.s_down;
   a.H = (int)c.s.H; a.I = (int)c.s.I; a.E = (int)c.s.E;
-  a.cap = (int)c.L.cap; a.tpe = (int)c.L.tpe;
+  a.tiles = c.L.tiles;
   a.xq_dt = c.s.xq_dtype; a.w_dt = c.s.weight_dtype; a.h_dt = c.s.h_dtype; a.y_dt = c.s.y_dtype;
   a.ws = c.ws;
   a.hsf = c.s.h_dtype == MOE_E4M3 ? c.ws.hsf : nullptr;

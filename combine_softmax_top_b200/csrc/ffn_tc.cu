@@ -92,6 +92,7 @@ struct TcParams {
   void* y;
   Ws ws;
   int H, I, E, cap, tpe;
+  int compact;               // expert windows start at base[e] tiles (set_base)
   int n_islices, n_hslices;  // I/128, H/128
   int nk1, nk2;              // K slabs of gate/up (over H) and down (over I)
   int kelems;                // elements per slab
@@ -152,17 +153,16 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_fla
   }
 }
 
-// Rows of tile `tile` of expert `e` once its sentinel carries this epoch.
-__device__ bool wait_tile(const TcParams& p, uint32_t epoch, int e, int tile, volatile int* abort_flag,
-                          int* rows) {
+// Rows of global tile g once its sentinel carries this epoch.
+__device__ bool wait_tile(const TcParams& p, uint32_t epoch, int g, volatile int* abort_flag, int* rows) {
   const unsigned long long t0 = globaltimer();
-  const uint32_t* sp = p.ws.sentinel + (int64_t)e * p.tpe + tile;
+  const uint32_t* sp = p.ws.sentinel + g;
   while (true) {
     const uint32_t s = ld_acquire(sp);
     if ((s >> 8) == (epoch & 0xFFFFFFu)) {
       *rows = (int)(s & 0xFF);
       if (*rows < 1 || *rows > kTileRows) {   // never published: a corrupt workspace
-        latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x22000000u | (uint32_t)(e * p.tpe + tile));
+        latch_error(p.ws.hdr, MOE_ERR_INVALID_ARG, 0x22000000u | (uint32_t)g);
         *abort_flag = 1;
         return false;
       }
@@ -170,7 +170,7 @@ __device__ bool wait_tile(const TcParams& p, uint32_t epoch, int e, int tile, vo
     }
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitBudgetNs) {
-      latch_error(p.ws.hdr, MOE_ERR_TIMEOUT, 0x23000000u | (uint32_t)(e * p.tpe + tile));
+      latch_error(p.ws.hdr, MOE_ERR_TIMEOUT, 0x23000000u | (uint32_t)g);
       *abort_flag = 1;
       return false;
     }
@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // expert's last tile of at most kTailMax rows joins the tile before it:
     // its weights are then not streamed again for a few tokens.
     int* chunk_tab = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1]
+    const uint32_t* base = p.compact ? set_base(set, p.E, p.tiles) : nullptr;
     int ntab = 0;   // tiles counted from the expert counts (lane 31)
     {
       const uint32_t* cnt = set_count(set);
@@ -369,13 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         j.pair = j.kind == kKindDown && dpair == 2;
         j.slice = (int)(w / nc) * (j.pair ? 2 : 1);
         j.tile = (int)(w % nc);
-        j.slot = j.e * p.tpe + j.tile;     // global tile id: the down units' counter
+        // global tile: rows 128 * slot ..., the down units' counter
+        j.slot = (base ? (int)base[j.e] : j.e * p.tpe) + j.tile;
         j.wide = tail && j.tile == (int)nc - 1;
         int rows = 0;
-        good = wait_tile(p, epoch, j.e, j.tile, abort_flag, &rows);
+        good = wait_tile(p, epoch, j.slot, abort_flag, &rows);
         if (good && j.wide) {   // the joined tail's sentinel too
           int rows2 = 0;
-          good = wait_tile(p, epoch, j.e, j.tile + 1, abort_flag, &rows2);
+          good = wait_tile(p, epoch, j.slot + 1, abort_flag, &rows2);
           rows += rows2;
         }
         if (!good) break;
@@ -428,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int N = (j.rows + 15) & ~15;
       const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
       const int arow = j.e * (down ? p.H : p.I) + j.slice * 128;
-      const int brow = j.e * p.cap + j.tile * kTileRows + j.row_off;
-      const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
+      const int brow = j.slot * kTileRows + j.row_off;
+      const int64_t tile_g = j.slot;
       const bool dual = !down || j.pair;   // two weight tiles share the token tile
       const uint32_t tx = (dual ? 2u : (uint32_t)j.nslab) * kABytes + (uint32_t)(j.nslab * N * kSlab);
       // the job's weight scales, one per 128 x 128 block along K: lane l holds
@@ -743,8 +745,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       while (!ptx::mbar_try_wait(acc_full + s0, (acc_ph >> s0) & 1u)) {}   // completed: returns at once
       if (two) while (!ptx::mbar_try_wait(acc_full + s1, (acc_ph >> s1) & 1u)) {}
       ptx::tc_fence_after();
-      const int64_t row0 = (int64_t)j.e * p.cap + (int64_t)j.tile * kTileRows + j.row_off;
-      const int64_t tile_g = (int64_t)j.e * p.tpe + j.tile;
+      const int64_t row0 = (int64_t)j.slot * kTileRows + j.row_off;
+      const int64_t tile_g = j.slot;
       // Set s owns the 32-token batches at columns 32 s and 32 s + 64 (a job
       // has at most 128 rows). Both are drained from TMEM into registers first
       // -- h = SwiGLU in fp32, or y already rounded to bf16 (two slices packed
@@ -929,7 +931,7 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   if (attr_err != cudaSuccess) return attr_err;
   TcParams p;
   memset(&p, 0, sizeof(p));
-  const int64_t H = c.s.H, I = c.s.I, E = c.s.E, rows = E * c.L.cap;
+  const int64_t H = c.s.H, I = c.s.I, E = c.s.E, rows = c.L.tiles * kTileRows;
   const int kel = kFp8 ? 128 : 64;
   if (!make_tmap(&p.tm_wg, w.w_gate, kFp8, H, E * I, kel, 128) ||
       !make_tmap(&p.tm_wu, w.w_up, kFp8, H, E * I, kel, 128) ||
@@ -952,6 +954,7 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.E = (int)E;
   p.cap = (int)c.L.cap;
   p.tpe = (int)c.L.tpe;
+  p.compact = c.L.compact ? 1 : 0;
   p.n_islices = (int)(I / 128);
   p.n_hslices = (int)(H / 128);
   p.kelems = kel;

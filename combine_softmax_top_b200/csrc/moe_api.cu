@@ -19,9 +19,12 @@ moe_status check_shape(const moe_shape* s) {
   if (!s) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->H <= 0 || s->E < 1 || s->E > 65535) return MOE_ERR_INVALID_ARG;
   if (s->topk < 1 || s->topk > s->E || s->topk > kMaxTopk) return MOE_ERR_INVALID_ARG;
-  if (s->quant_block != kQBlock || (s->flags & ~MOE_FLAG_SHARED_EXPERT) != 0) return MOE_ERR_INVALID_ARG;
+  if (s->quant_block != kQBlock || (s->flags & ~(MOE_FLAG_SHARED_EXPERT | MOE_FLAG_COMPACT)) != 0)
+    return MOE_ERR_INVALID_ARG;
   const bool shared = (s->flags & MOE_FLAG_SHARED_EXPERT) != 0;
-  if (shared && (s->identity_experts || s->topk + 1 > kMaxTopk || s->E + 1 > 65535 || default_cap(*s) < s->T))
+  const bool compact = (s->flags & MOE_FLAG_COMPACT) != 0;
+  if (shared && (s->identity_experts || s->topk + 1 > kMaxTopk || s->E + 1 > 65535 ||
+                 (!compact && default_cap(*s) < s->T)))
     return MOE_ERR_INVALID_ARG;   // the shared expert takes every token
   if ((s->renorm != 0 && s->renorm != 1) || (s->identity_experts != 0 && s->identity_experts != 1))
     return MOE_ERR_INVALID_ARG;
@@ -32,10 +35,15 @@ moe_status check_shape(const moe_shape* s) {
     return MOE_ERR_INVALID_ARG;
   if (s->act_dtype == MOE_E4M3 || s->out_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (s->xq_dtype == MOE_E4M3 && s->H % kQBlock != 0) return MOE_ERR_INVALID_ARG;
-  const int64_t cap = default_cap(*s);
   const int64_t ne = s->E + (shared ? 1 : 0), nk = s->topk + (shared ? 1 : 0);
-  if (cap / kTileRows > 65535 || ne * cap >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
   if (s->T * nk >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (compact) {
+    // windows sized by the counting pass; tile ids fit 16 bits per expert
+    if (s->cap_rows != 0 || ceil_div(s->T * nk, kTileRows) + ne > 65535) return MOE_ERR_INVALID_ARG;
+  } else {
+    const int64_t cap = default_cap(*s);
+    if (cap / kTileRows > 65535 || ne * cap >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  }
   if (s->identity_experts) return MOE_OK;
   if (s->I <= 0 || s->I > (1 << 24) || s->I % 16 != 0) return MOE_ERR_INVALID_ARG;
   if (!is_dtype(s->weight_dtype) || !is_dtype(s->h_dtype) || !is_dtype(s->y_dtype))

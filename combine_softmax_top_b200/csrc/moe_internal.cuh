@@ -24,12 +24,17 @@ constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
 //
 // header : epoch_next, epoch_cur, error, error_info (u32 each)
 // set    : misc[8] (ring_head, done, ring_total, ...) | count[E] |
-//          fill[E*tpe] | hdone[E*tpe]
+//          fill[tiles] | hdone[tiles] | pre[E] | base[E + 1]
 //          two sets are used alternately by consecutive dispatches; each
 //          dispatch zeroes the set the following dispatch will use.
-//          hdone[slot] counts the finished gate/up slices of ring slot `slot`.
-// sentinel[E*tpe] u32 : (epoch << 8) | rows of a published tile
-// ring[E*tpe] u64     : (epoch << 32) | (e << 16) | tile, in publication order
+//          hdone[g] counts the finished gate/up slices of global tile g;
+//          pre / base: compact windows only (expert pair counts taken before
+//          dispatch, and each expert's first global tile).
+// A global tile g covers rows 128 g .. 128 g + 127 of the expert buffers:
+// expert e's tile i is g = e * tpe + i (windows of cap rows) or base[e] + i
+// (compact windows); tiles = E * tpe or the compact bound.
+// sentinel[tiles] u32 : (epoch << 8) | rows of a published tile
+// ring[tiles] u64     : (epoch mod 2^24) << 40 | e << 24 | g, in publication order
 // xsf / hsf           : UE8M0 scale atoms of xq / hq for the block-scaled MMA,
 //                       [tile][group of four 128-value blocks][512 B]; row m of
 //                       the tile owns the 32-bit word at (m % 32) * 16 +
@@ -43,10 +48,11 @@ struct Header {
 };
 static_assert(sizeof(Header) == 256, "header size");
 
-enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kMiscWords = 8 };
+enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kPlanDone = 6, kMiscWords = 8 };
 
 struct Layout {
-  int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles = E * tpe
+  int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles: E * tpe, or the compact bound
+  bool compact;                             // windows packed at offsets[e] (MOE_FLAG_COMPACT)
   int64_t hgroups, igroups;                 // ceil(H/512), ceil(I/512): scale atoms per tile
   size_t set_words;                         // u32 words of one counter set
   size_t off_set[2], off_sentinel, off_ring, off_xsf, off_hsf, total;
@@ -64,12 +70,21 @@ inline int64_t default_cap(const moe_shape& s) {
 inline Layout make_layout(const moe_shape& s) {
   Layout L{};
   L.T = s.T; L.H = s.H; L.E = s.E; L.k = s.topk; L.I = s.I;
-  L.cap = default_cap(s);
-  L.tpe = ceil_div(L.cap, kTileRows);
-  L.tiles = L.E * L.tpe;
+  L.compact = (s.flags & MOE_FLAG_COMPACT) != 0;
+  if (L.compact) {
+    // windows rounded up to whole tiles: the T * k rows plus at most one
+    // partial tile per expert
+    L.tiles = ceil_div(L.T * L.k, kTileRows) + L.E;
+    L.cap = L.tiles * kTileRows;   // no per-expert limit
+    L.tpe = L.tiles;
+  } else {
+    L.cap = default_cap(s);
+    L.tpe = ceil_div(L.cap, kTileRows);
+    L.tiles = L.E * L.tpe;
+  }
   L.hgroups = ceil_div(L.H, 4 * kQBlock);
   L.igroups = ceil_div(L.I, 4 * kQBlock);
-  L.set_words = (size_t)(kMiscWords + L.E + 2 * L.tiles);
+  L.set_words = (size_t)(kMiscWords + L.E + 2 * L.tiles + 2 * L.E + 1);
   size_t off = sizeof(Header);
   for (int i = 0; i < 2; ++i) {
     L.off_set[i] = off;
@@ -191,6 +206,20 @@ __device__ __forceinline__ uint32_t* set_count(uint32_t* set) { return set + kMi
 __device__ __forceinline__ uint32_t* set_fill(uint32_t* set, int E) { return set + kMiscWords + E; }
 __device__ __forceinline__ uint32_t* set_hdone(uint32_t* set, int E, int64_t tiles) {
   return set + kMiscWords + E + tiles;
+}
+// compact windows: each expert's pair count, and its first global tile
+// (entry E: the tiles of all windows), both written before dispatch
+__device__ __forceinline__ uint32_t* set_pre(uint32_t* set, int E, int64_t tiles) {
+  return set + kMiscWords + E + 2 * tiles;
+}
+__device__ __forceinline__ uint32_t* set_base(uint32_t* set, int E, int64_t tiles) {
+  return set + kMiscWords + 2 * E + 2 * tiles;
+}
+
+// Ring entries: 24 bits of epoch (as the sentinels), expert, global tile.
+__device__ __forceinline__ unsigned long long ring_entry(uint32_t epoch, int e, int64_t g) {
+  return ((unsigned long long)(epoch & 0xFFFFFFu) << 40) | ((unsigned long long)e << 24) |
+         (unsigned long long)g;
 }
 
 // ---- host-side argument checks (moe_api.cu) ---------------------------------

@@ -118,7 +118,8 @@ def make_shape(s: Spec, T: int | None = None) -> moe_shape:
     sh.weight_dtype, sh.h_dtype, sh.y_dtype, sh.out_dtype = _DT[s.weight], _DT[s.h], _DT[s.y], _DT[s.out]
     sh.renorm, sh.identity_experts = s.renorm, s.identity
     sh.cap_rows = s.cap_rows
-    sh.quant_block, sh.flags = 128, (1 if s.shared else 0)   # 1: MOE_FLAG_SHARED_EXPERT
+    # MOE_FLAG_SHARED_EXPERT = 1, MOE_FLAG_COMPACT = 2
+    sh.quant_block, sh.flags = 128, (1 if s.shared else 0) | (2 if s.compact else 0)
     return sh
 
 
@@ -216,9 +217,8 @@ def alloc_buffers(s: Spec, device="cuda", T: int | None = None, stream=None) -> 
     the workspace."""
     sh = make_shape(s, T)
     T = sh.T
-    cap = s.cap_rows if s.cap_rows else max(128, -(-T // 128) * 128)
     ne, ks = s.E + s.shared, s.k + s.shared   # a shared expert adds one expert and one slot
-    rows = ne * cap
+    rows = s.rows(T)
     nws = moe_workspace_bytes(sh)
     ws = torch.empty(nws, dtype=torch.uint8, device=device)
     z = dict(device=device)

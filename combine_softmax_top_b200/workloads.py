@@ -48,6 +48,7 @@ class Spec:
     zipf_s: float = 0.0   # > 0: add log p_e, p_e proportional to (e+1)^-s, to the logits
     cap_rows: int = 0     # 0: default round_up(T, 128)
     shared: int = 0       # 1: one shared expert (index E) every token also goes through, weight 1
+    compact: int = 0      # 1: expert windows packed back to back after a counting pass
     extra: dict = field(default_factory=dict)
 
     def with_(self, **kw) -> "Spec":
@@ -66,6 +67,15 @@ class Spec:
     def ks(self) -> int:
         """Slots per token (the shared expert's included)."""
         return self.k + self.shared
+
+    def rows(self, T: int | None = None) -> int:
+        """Rows of the expert buffers: ne windows of cap rows, or with compact
+        windows the T * ks pairs plus one partial 128-row tile per expert."""
+        T = self.T if T is None else T
+        if self.compact:
+            return (-(-T * self.ks // 128) + self.ne) * 128
+        cap = self.cap_rows if self.cap_rows else max(128, -(-T // 128) * 128)
+        return self.ne * cap
 
 
 # The five workloads of the layer (tiny fp32, decode, prefill, skewed routing,

@@ -102,6 +102,19 @@ typedef enum moe_status {
  */
 enum { MOE_FLAG_SHARED_EXPERT = 1 };
 
+/*
+ * flags |= MOE_FLAG_COMPACT packs the expert windows instead of giving every
+ * expert cap rows: moe_dispatch first counts each expert's pairs (a fence:
+ * the counts are complete before any row is placed, the NVLinkOneSided
+ * abstract's Fence protocol), then expert e's window starts at offsets[e], the
+ * 128-row-aligned running sum of the windows before it, and holds exactly
+ * counts[e] rows (no capacity limit, no overflow). rows = 128 *
+ * (ceil(T * slots / 128) + experts), slots = topk (+ 1 with a shared
+ * expert), experts = E (+ 1); rows / 128 <= 65535. cap_rows must be 0.
+ * moe_dispatch_noalloc returns MOE_ERR_UNSUPPORTED for it.
+ */
+enum { MOE_FLAG_COMPACT = 2 };
+
 typedef struct moe_shape {
   int64_t T;              /* tokens, >= 0 */
   int64_t H;              /* hidden size */
@@ -118,17 +131,18 @@ typedef struct moe_shape {
   int32_t identity_experts; /* 1: every expert returns its input (no FFN) */
   int64_t cap_rows;       /* rows per expert window; 0 = round_up(T, 128) */
   int32_t quant_block;    /* must be 128 */
-  int32_t flags;          /* 0, or MOE_FLAG_SHARED_EXPERT */
+  int32_t flags;          /* 0 or MOE_FLAG_SHARED_EXPERT | MOE_FLAG_COMPACT */
 } moe_shape;
 
 /*
  * Expert-major buffers written by moe_dispatch and moe_grouped_ffn (all device,
  * caller-owned). cap = cap_rows (or its default); rows = E * cap. Expert e owns
- * rows [e * cap, e * cap + counts[e]).
+ * rows [offsets[e], offsets[e] + counts[e]) (offsets[e] = e * cap, or packed
+ * with MOE_FLAG_COMPACT, which also sets rows).
  *   xq      [rows, H]        tokens in xq_dtype
  *   xs      [rows, H/128]    fp32 power-of-two scales (E4M3 xq only, else NULL)
  *   counts  [E]   int32      rows filled per expert (bit-exact routing counts)
- *   offsets [E]   int32      first row of each expert window (= e * cap)
+ *   offsets [E]   int32      first row of each expert window (e * cap, or packed)
  *   row_src [rows] int32     row -> pair id t*topk + j (rows past counts[e]
  *                            are left as they were)
  *   pos     [T*topk] int32   pair id -> row, or -1 if it was not placed
@@ -202,7 +216,7 @@ MOE_API moe_status moe_route(const moe_shape* shape, const float* logits, int32_
  *   topk_idx [T, topk] int32, device (experts must be in [0, E) and distinct
  *            per token)
  *   bufs     xq, xs, counts, offsets, row_src, pos are written
- * Each pair claims row e*cap + atomicAdd(count[e], 1); E4M3 rows are
+ * Each pair claims row offsets[e] + atomicAdd(count[e], 1); E4M3 rows are
  * quantised per 128 values with the smallest power-of-two scale that keeps
  * the block within +-448. A pair that finds its expert full is not placed,
  * pos = -1, and MOE_ERR_CAPACITY is latched. Every completed 128-row tile
@@ -220,7 +234,7 @@ MOE_API moe_status moe_dispatch(const moe_shape* shape, const void* x, const int
  *   y_r = h W_down[e]^T, stored as y_dtype.
  *   bufs  dispatch outputs (read) and hq/hs (written)
  *   w     expert weights
- *   y     [E*cap, H] y_dtype, device (out; rows past counts[e] untouched)
+ *   y     [rows, H] y_dtype, device (out; rows past counts[e] untouched)
  * Work starts per tile as its sentinel is found set; waits are bounded and
  * latch MOE_ERR_TIMEOUT.
  */
@@ -235,7 +249,7 @@ MOE_API moe_status moe_grouped_ffn(const moe_shape* shape, const moe_dispatch_bu
  * experts the rows are the dispatched tokens themselves (xq, dequantised with
  * xs) and y may be NULL. Pairs with pos = -1 contribute nothing.
  *   bufs   pos (and xq/xs for identity experts)
- *   y      [E*cap, H] y_dtype, device
+ *   y      [rows, H] y_dtype, device
  *   topk_w [T, topk] fp32, device
  *   out    [T, H] out_dtype, device
  */

@@ -49,11 +49,22 @@ def oracle_problem(s: W.Spec, inp: dict, experts=None) -> oracle.Problem:
     return oracle.Problem(s.T, s.H, s.E, s.k, s.I, **kw)
 
 
+def window_offsets(s: W.Spec, counts: np.ndarray) -> np.ndarray:
+    """First row of each expert window: e * cap, or with compact windows the
+    running sum of the windows before it, each rounded up to 128 rows (the
+    layout moe.h states for MOE_FLAG_COMPACT)."""
+    if not s.compact:
+        return np.arange(len(counts), dtype=np.int64) * s.cap
+    tiles = -(-counts.astype(np.int64) // 128)
+    return 128 * np.concatenate([[0], np.cumsum(tiles)[:-1]])
+
+
 def placed_rows(b: moe.Buffers):
-    """(row ids, pair ids, expert ids) of every filled row, from counts/row_src."""
+    """(row ids, pair ids, expert ids) of every filled row, from counts,
+    offsets and row_src."""
     counts = b.counts.cpu().numpy()
-    cap = b.xq.shape[0] // b.spec.ne
-    rows = np.concatenate([e * cap + np.arange(c) for e, c in enumerate(counts)]) if counts.sum() \
+    offsets = b.offsets.cpu().numpy().astype(np.int64)
+    rows = np.concatenate([o + np.arange(c) for o, c in zip(offsets, counts)]) if counts.sum() \
         else np.zeros(0, np.int64)
     experts = np.repeat(np.arange(b.spec.ne), counts)
     pairs = b.row_src.cpu().numpy()[rows]

@@ -49,7 +49,7 @@ def test_workspace_grows_with_capacity():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("topk", 0), ("topk", 33), ("E", 0), ("H", 100), ("quant_block", 64), ("flags", 2),
+    ("topk", 0), ("topk", 33), ("E", 0), ("H", 100), ("quant_block", 64), ("flags", 4),
     ("cap_rows", 100), ("renorm", 2), ("T", -1), ("act_dtype", 7),
 ])
 def test_invalid_shapes_rejected_on_host(field, value):
@@ -85,6 +85,31 @@ def test_shared_expert_workspace_covers_one_more_expert():
     assert b > a
 
 
+@pytest.mark.parametrize("over", [
+    {"cap_rows": 128},   # the counting pass sizes the windows
+    {"T": 1 << 20},      # more than 65535 tiles of 128 rows
+])
+def test_compact_windows_preconditions(over):
+    sh = moe.make_shape(W.spec("prefill", compact=1))
+    for f, v in over.items():
+        setattr(sh, f, v)
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 1
+
+
+def test_compact_windows_rows_and_workspace():
+    """Compact windows: the buffers hold T * k rows plus one partial tile per
+    expert instead of E windows of round_up(T, 128) rows; the workspace's
+    per-tile arrays shrink with them."""
+    s = W.spec("prefill")
+    c = s.with_(compact=1)
+    assert c.rows() == (8192 * 8 // 128 + 256) * 128 < s.rows() // 20
+    assert moe.moe_workspace_bytes(moe.make_shape(c)) < moe.moe_workspace_bytes(moe.make_shape(s))
+    sc = c.with_(shared=1)
+    assert sc.rows() == (-(-8192 * 9 // 128) + 257) * 128
+    assert moe.moe_workspace_bytes(moe.make_shape(sc)) > 0
+
+
 def test_unsupported_dtype_combination():
     sh = moe.make_shape(W.spec("decode"))
     sh.h_dtype = moe.MOE_BF16   # fp8 weights with a bf16 h is not a supported layer
@@ -98,3 +123,10 @@ def test_null_shape_and_output():
     sh = moe.make_shape(W.spec("tiny"))
     assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), None) == 1
     assert moe.lib().moe_poll_status(None, None) == 1
+
+
+def test_noalloc_dispatch_refuses_compact_windows():
+    """The no-workspace dispatch has no room for the counting pass: the
+    compact flag is refused before any pointer is looked at."""
+    sh = moe.make_shape(W.spec("decode", compact=1))
+    assert moe.lib().moe_dispatch_noalloc(ctypes.byref(sh), None, None, None, None) == 2

@@ -91,8 +91,7 @@ def test_dispatch_parity(name):
     counts = b.counts.cpu().numpy()
     assert np.array_equal(counts, oracle.counts(idx, s.E))
     assert counts.sum() == s.T * s.k
-    cap = s.cap
-    assert np.array_equal(b.offsets.cpu().numpy(), np.arange(s.E) * cap)
+    assert np.array_equal(b.offsets.cpu().numpy(), G.window_offsets(s, counts))
     rows, pairs, experts = G.placed_rows(b)
     # every pair placed exactly once, in its own expert's window
     assert np.array_equal(np.sort(pairs), np.arange(s.T * s.k))
@@ -258,7 +257,7 @@ def test_ffn_wait_runs_out_and_context_survives(cuda_device):
     hdr = b.ws[:16].view(torch.int32)
     assert int(hdr[1]) == 1
     tpe = s.cap // 128
-    set_words = 8 + s.E + 2 * s.E * tpe
+    set_words = 8 + s.E + 2 * s.E * tpe + 2 * s.E + 1
     sent_off = 256 + 2 * (((set_words * 4 + 255) // 256) * 256)
     sentinels = b.ws[sent_off:sent_off + 4 * s.E * tpe].view(torch.int32)
     e = int(np.nonzero(b.counts.cpu().numpy())[0][0])
