@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.cpp")
 LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
-F32, BF16, E4M3 = 0, 1, 2
+F32, BF16, E4M3, E2M1 = 0, 1, 2, 3
 OK, BAD_ARG, NONFINITE = 0, 1, 6
 
 
@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         sigs = {
             "oracle_e4m3_encode": [P, P, I64],
             "oracle_e4m3_decode": [P, P, I64],
+            "oracle_e2m1_decode": [P, P, I64],
+            "oracle_ue8m0_decode": [P, P, I64],
             "oracle_bf16_round": [P, P, I64],
             "oracle_pow2_scale": [P, P, I64],
             "oracle_route": [I64, I64, I64, I32, P, P, P],
@@ -113,8 +115,10 @@ class Problem:
     """Shapes, dtypes and expert weights of one MoE layer.
 
     Weights are either full arrays ([E, I, H] gate/up, [E, H, I] down, e4m3
-    scales [E, I/128, H/128] / [E, H/128, I/128]) or mappings from expert index
-    to that expert's matrix, for checks that touch only a few experts. With
+    scales [E, I/128, H/128] / [E, H/128, I/128]; e2m1 weights packed two per
+    byte, [E, I, H/2] / [E, H, I/2], element 2i in the low nibble, with UE8M0
+    scale bytes [E, I, H/32] / [E, H, I/32]) or mappings from expert index to
+    that expert's matrix, for checks that touch only a few experts. With
     shared=1 the arrays hold E + 1 experts: expert E is the shared expert that
     every token also goes through, added with weight 1.
     """
@@ -177,6 +181,22 @@ def e4m3_decode(q: np.ndarray) -> np.ndarray:
     q = np.ascontiguousarray(q, dtype=np.uint8)
     out = np.empty(q.shape, np.float64)
     _call("oracle_e4m3_decode", _ptr(q), _ptr(out), q.size)
+    return out
+
+
+def e2m1_decode(q: np.ndarray) -> np.ndarray:
+    """4-bit E2M1 codes (one per uint8, low nibble) -> float64 values."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    out = np.empty(q.shape, np.float64)
+    _call("oracle_e2m1_decode", _ptr(q), _ptr(out), q.size)
+    return out
+
+
+def ue8m0_decode(b: np.ndarray) -> np.ndarray:
+    """UE8M0 scale bytes -> float64 powers of two (255 -> NaN)."""
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(b.shape, np.float64)
+    _call("oracle_ue8m0_decode", _ptr(b), _ptr(out), b.size)
     return out
 
 

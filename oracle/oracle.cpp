@@ -22,6 +22,10 @@
 //    "Two MMA Implementations"). The pages print a 32-element block; this build
 //    uses 128-element blocks with power-of-two fp32 scales, which the same
 //    block-scaled MMA consumes exactly.
+//  * 4-bit weights are the microscaling (MX) form the same paragraph names:
+//    every 32 consecutive elements share one exponent scale, and the weights
+//    shrink to 4 bits. Read as the OCP MX formats: FP4 E2M1 elements with one
+//    UE8M0 scale (2^(byte - 127)) per 32 elements along K.
 //  * Combine weights each expert output by its routing weight and sums back in
 //    token order (NVLinkOneSided abstract; Ascend report abstract, "direct
 //    reading from remote expert windows").
@@ -46,7 +50,7 @@
 extern "C" {
 
 // dtype codes used by this oracle's own entry points
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2, ORC_E2M1 = 3 };
 
 enum {
   ORC_OK = 0,
@@ -67,15 +71,17 @@ typedef struct oracle_problem {
   int32_t shared;     // 1: expert E is a shared expert every token also goes
                       //    through, added with weight 1 after the k routed ones
   // One pointer per expert (E + shared entries each). Expert e's matrices are
-  // row-major: gate/up [I, H], down [H, I]; e4m3 scales [I/128, H/128] and
-  // [H/128, I/128]. A NULL entry marks an expert whose weights were not
-  // provided; using it is an error.
+  // row-major: gate/up [I, H], down [H, I]; e4m3 scales fp32 [I/128, H/128]
+  // and [H/128, I/128]. e2m1 weights hold two elements per byte (element 2i
+  // in the low nibble of byte i of its row) with UE8M0 scale bytes
+  // [I, H/32] and [H, I/32]. A NULL entry marks an expert whose weights were
+  // not provided; using it is an error.
   const void* const* w_gate;
   const void* const* w_up;
   const void* const* w_down;
-  const float* const* s_gate;  // e4m3 weights only
-  const float* const* s_up;
-  const float* const* s_down;
+  const void* const* s_gate;  // e4m3 and e2m1 weights only
+  const void* const* s_up;
+  const void* const* s_down;
 } oracle_problem;
 
 // ---------------------------------------------------------------- formats --
@@ -117,6 +123,23 @@ static uint8_t e4m3_code(double v) {
   int code = ((exp2 + 7) << 3) | (int)mant;
   if (code > 0x7E) code = 0x7E;
   return sign | (uint8_t)code;
+}
+
+// OCP MX FP4, E2M1: 1 sign bit (bit 3), 2 exponent bits with bias 1, 1
+// mantissa bit; exponent field 0 holds the subnormal m * 2^-1. No infinity
+// or NaN: the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+static double e2m1_value(uint8_t code) {
+  const int sign = (code >> 3) & 1;
+  const int ef = (code >> 1) & 3;
+  const int mf = code & 1;
+  const double mag = ef == 0 ? 0.5 * mf : std::ldexp(1.0 + 0.5 * mf, ef - 1);
+  return sign ? -mag : mag;
+}
+
+// OCP MX UE8M0 scale: 2^(byte - 127); the byte 255 is NaN.
+static double ue8m0_value(uint8_t b) {
+  if (b == 255) return std::nan("");
+  return std::ldexp(1.0, (int)b - 127);
 }
 
 // bfloat16: the upper 16 bits of an IEEE binary32.
@@ -173,6 +196,17 @@ int oracle_e4m3_encode(const double* v, uint8_t* out, int64_t n) {
 
 int oracle_e4m3_decode(const uint8_t* q, double* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(q[i]);
+  return ORC_OK;
+}
+
+// 4-bit E2M1 codes (one per byte, low nibble) and UE8M0 scale bytes to doubles
+int oracle_e2m1_decode(const uint8_t* q, double* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e2m1_value(q[i] & 15);
+  return ORC_OK;
+}
+
+int oracle_ue8m0_decode(const uint8_t* b, double* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = ue8m0_value(b[i]);
   return ORC_OK;
 }
 
@@ -258,19 +292,26 @@ static double load_act(const void* p, int32_t dt, int64_t i) {
 }
 
 // element [r, c] of one expert's weight matrix of shape [rows, cols]
-static inline double weight_at(const void* w, const float* s, int32_t dt,
+static inline double weight_at(const void* w, const void* s, int32_t dt,
                                int64_t cols, int64_t r, int64_t c) {
   const int64_t off = r * cols + c;
   if (dt == ORC_F32) return (double)((const float*)w)[off];
   if (dt == ORC_BF16) return bf16_value(((const uint16_t*)w)[off]);
-  const double sc = (double)s[(r / 128) * (cols / 128) + c / 128];
+  if (dt == ORC_E2M1) {
+    const uint8_t byte = ((const uint8_t*)w)[r * (cols / 2) + c / 2];
+    const uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+    return e2m1_value(code) * ue8m0_value(((const uint8_t*)s)[r * (cols / 32) + c / 32]);
+  }
+  const double sc = (double)((const float*)s)[(r / 128) * (cols / 128) + c / 128];
   return e4m3_value(((const uint8_t*)w)[off]) * sc;
 }
+
+static bool scaled_weights(int32_t dt) { return dt == ORC_E4M3 || dt == ORC_E2M1; }
 
 static bool have_expert(const oracle_problem* p, int64_t e) {
   if (e < 0 || e >= p->E + (p->shared ? 1 : 0)) return false;
   if (!p->w_gate[e] || !p->w_up[e] || !p->w_down[e]) return false;
-  if (p->w_dtype == ORC_E4M3 && (!p->s_gate[e] || !p->s_up[e] || !p->s_down[e])) return false;
+  if (scaled_weights(p->w_dtype) && (!p->s_gate[e] || !p->s_up[e] || !p->s_down[e])) return false;
   return true;
 }
 
@@ -282,13 +323,13 @@ static double silu(double g) { return g / (1.0 + std::exp(-g)); }
 static void expert_row(const oracle_problem* p, int64_t e, const double* xh,
                        void* h_raw, float* hs, void* y_raw, double* yd) {
   const int64_t H = p->H, I = p->I;
-  const bool e4 = p->w_dtype == ORC_E4M3;
+  const bool scaled = scaled_weights(p->w_dtype);
   const void* wg = p->w_gate[e];
   const void* wu = p->w_up[e];
   const void* wd = p->w_down[e];
-  const float* sg = e4 ? p->s_gate[e] : nullptr;
-  const float* su = e4 ? p->s_up[e] : nullptr;
-  const float* sd = e4 ? p->s_down[e] : nullptr;
+  const void* sg = scaled ? p->s_gate[e] : nullptr;
+  const void* su = scaled ? p->s_up[e] : nullptr;
+  const void* sd = scaled ? p->s_down[e] : nullptr;
   std::vector<float> h32(I);
   std::vector<double> hh(I);
   for (int64_t i = 0; i < I; ++i) {
@@ -367,6 +408,7 @@ static int check_problem(const oracle_problem* p) {
   if (p->xq_dtype == ORC_E4M3 && p->H % 128) return ORC_BAD_ARG;
   if (p->h_dtype == ORC_E4M3 && p->I % 128) return ORC_BAD_ARG;
   if (p->w_dtype == ORC_E4M3 && (p->H % 128 || p->I % 128)) return ORC_BAD_ARG;
+  if (p->w_dtype == ORC_E2M1 && (p->H % 32 || p->I % 32)) return ORC_BAD_ARG;
   return ORC_OK;
 }
 

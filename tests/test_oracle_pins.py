@@ -469,3 +469,129 @@ def test_shared_expert_alone_is_the_dense_ffn():
     yp = r["y_pairs"].reshape(s.T, s.k + 1, s.H)
     assert max_abs_rel(yp[:, s.k], ref.numpy()) < 1e-6
     assert np.all(yp[:, : s.k] == 0)
+
+
+# ---------------------------------------------------- MX FP4 (E2M1) weights --
+
+# OCP Microscaling Formats (MX) v1.0, FP4 E2M1: the eight magnitudes the
+# format represents (codes 0-7; codes 8-15 are their negatives).
+_E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_all_codes():
+    got = oracle.e2m1_decode(np.arange(16, dtype=np.uint8))
+    ref = np.array(_E2M1_TABLE + [-v for v in _E2M1_TABLE])
+    assert np.array_equal(got, ref)
+    assert np.signbit(got[8])   # code 8 is -0
+
+
+def test_ue8m0_decode():
+    """UE8M0 (MX v1.0): 2^(byte - 127), byte 255 is NaN."""
+    got = oracle.ue8m0_decode(np.array([0, 1, 126, 127, 128, 254, 255], np.uint8))
+    assert got[0] == 2.0 ** -127 and got[1] == 2.0 ** -126
+    assert got[2] == 0.5 and got[3] == 1.0 and got[4] == 2.0 and got[5] == 2.0 ** 127
+    assert np.isnan(got[6])
+
+
+def _random_mxfp4(rng, rows, cols):
+    """Random packed E2M1 codes (two per byte) and UE8M0 scales per 32."""
+    packed = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+    scales = rng.integers(118, 124, size=(rows, cols // 32), dtype=np.uint8)
+    return packed, scales
+
+
+def _dequant_mxfp4(packed, scales):
+    """Independent decode: element 2i is the low nibble of byte i, 2i + 1 the
+    high one; every 32 consecutive elements of a row share one scale."""
+    table = np.array(_E2M1_TABLE + [-v for v in _E2M1_TABLE])
+    rows = packed.shape[0]
+    codes = np.empty((rows, packed.shape[1] * 2), np.uint8)
+    codes[:, 0::2] = packed & 15
+    codes[:, 1::2] = packed >> 4
+    sc = np.repeat(np.exp2(scales.astype(np.float64) - 127.0), 32, axis=1)
+    return torch.from_numpy(table[codes] * sc)
+
+
+def _fp4_problem(T, H, E, I, wg, wu, wd, sg, su, sd):
+    return oracle.Problem(T, H, E, 1, I, x_dtype=oracle.BF16, xq_dtype=oracle.E4M3,
+                          w_dtype=oracle.E2M1, h_dtype=oracle.E4M3, y_dtype=oracle.BF16,
+                          out_dtype=oracle.BF16, w_gate=wg, w_up=wu, w_down=wd,
+                          s_gate=sg, s_up=su, s_down=sd)
+
+
+def test_expert_rows_e2m1_matches_torch():
+    """MX FP4 weights (GC-MoE explainer, "Two MMA Implementations": 4-bit
+    weights, one shared exponent per 32 elements): the oracle's expert rows
+    equal a float64 torch FFN over independently decoded weights."""
+    rng = np.random.default_rng(7)
+    T, H, E, I = 5, 256, 2, 384
+    wg, sg = zip(*[_random_mxfp4(rng, I, H) for _ in range(E)])
+    wu, su = zip(*[_random_mxfp4(rng, I, H) for _ in range(E)])
+    wd, sd = zip(*[_random_mxfp4(rng, H, I) for _ in range(E)])
+    st = lambda a: np.ascontiguousarray(np.stack(a))
+    p = _fp4_problem(T, H, E, I, st(wg), st(wu), st(wd), st(sg), st(su), st(sd))
+    x32 = rng.standard_normal((T, H)).astype(np.float32)
+    xq, xs = oracle.quantize_rows(x32)
+    experts = np.array([0, 1, 1, 0, 1], np.int32)
+    h, hs, y = oracle.expert_rows(p, experts, xq, xs)
+    xh = torch.from_numpy(xq).view(torch.float8_e4m3fn).double() * \
+        torch.from_numpy(xs).double().repeat_interleave(128, 1)
+    for r in range(T):
+        e = experts[r]
+        rh, ry = _dense_ffn_torch(xh[r:r + 1], _dequant_mxfp4(wg[e], sg[e]), _dequant_mxfp4(wu[e], su[e]),
+                                  _dequant_mxfp4(wd[e], sd[e]), _torch_requant, _torch_bf16)
+        hv = oracle.e4m3_decode(h[r]) * np.repeat(hs[r].astype(np.float64), 128)
+        assert np.array_equal(hv, rh[0].numpy())
+        assert max_abs_rel(bf16_bits_to_f32(y[r]), ry[0].numpy()) < 2 ** -7
+
+
+def test_e2m1_weights_equal_e4m3_weights_with_one_scale_per_block():
+    """Every E2M1 value is an E4M3 value. With one UE8M0 scale per 128 x 128
+    block, the FP4 expert must give the same bytes as the E4M3 expert holding
+    the same values with the equal fp32 block scales (two decode paths)."""
+    rng = np.random.default_rng(9)
+    T, H, I = 4, 256, 256
+    mats = {}
+    for name, (r, c) in (("g", (I, H)), ("u", (I, H)), ("d", (H, I))):
+        packed, _ = _random_mxfp4(rng, r, c)
+        blk = rng.integers(119, 123, size=(r // 128, c // 128), dtype=np.uint8)
+        s32 = np.repeat(np.repeat(blk, 128, 0), 4, 1)             # [r, c/32], constant per block
+        vals = _dequant_mxfp4(packed, np.full_like(s32, 127)).numpy()   # unscaled E2M1 values
+        codes = torch.from_numpy(vals).float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy(), vals)
+        mats[name] = (packed, s32, codes, np.exp2(blk.astype(np.float64) - 127).astype(np.float32))
+    x32 = rng.standard_normal((T, H)).astype(np.float32)
+    xq, xs = oracle.quantize_rows(x32)
+    experts = np.zeros(T, np.int32)
+    p4 = _fp4_problem(T, H, 1, I, *[mats[n][0][None] for n in "gud"], *[mats[n][1][None] for n in "gud"])
+    p8 = oracle.Problem(T, H, 1, 1, I, x_dtype=oracle.BF16, xq_dtype=oracle.E4M3, w_dtype=oracle.E4M3,
+                        h_dtype=oracle.E4M3, y_dtype=oracle.BF16, out_dtype=oracle.BF16,
+                        w_gate=mats["g"][2][None], w_up=mats["u"][2][None], w_down=mats["d"][2][None],
+                        s_gate=mats["g"][3][None], s_up=mats["u"][3][None], s_down=mats["d"][3][None])
+    h4, hs4, y4 = oracle.expert_rows(p4, experts, xq, xs)
+    h8, hs8, y8 = oracle.expert_rows(p8, experts, xq, xs)
+    assert np.array_equal(h4, h8) and np.array_equal(hs4, hs8) and np.array_equal(y4, y8)
+    assert np.abs(bf16_bits_to_f32(y4)).max() > 0
+
+
+def test_e2m1_nibble_order_and_scale_index_matter():
+    """Swapping the two nibbles of every byte, or transposing which 32-block a
+    scale belongs to, must change the result (guards the layout reading)."""
+    rng = np.random.default_rng(11)
+    T, H, I = 2, 128, 128
+    wg, sg = _random_mxfp4(rng, I, H)
+    wu, su = _random_mxfp4(rng, I, H)
+    wd, sd = _random_mxfp4(rng, H, I)
+    x32 = rng.standard_normal((T, H)).astype(np.float32)
+    xq, xs = oracle.quantize_rows(x32)
+    ex = np.zeros(T, np.int32)
+    base = oracle.expert_rows(_fp4_problem(T, H, 1, I, wg[None], wu[None], wd[None], sg[None], su[None], sd[None]),
+                              ex, xq, xs)[2]
+    swap = lambda b: ((b & 15) << 4) | (b >> 4)
+    swapped = oracle.expert_rows(_fp4_problem(T, H, 1, I, swap(wg)[None], wu[None], wd[None], sg[None], su[None],
+                                              sd[None]), ex, xq, xs)[2]
+    rolled = oracle.expert_rows(_fp4_problem(T, H, 1, I, wg[None], wu[None], wd[None],
+                                             np.ascontiguousarray(np.roll(sg, 1, axis=1))[None], su[None], sd[None]),
+                                ex, xq, xs)[2]
+    assert not np.array_equal(base, swapped)
+    assert not np.array_equal(base, rolled)
