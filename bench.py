@@ -301,6 +301,11 @@ def run_reference(args):
 
 
 EL = {"f32": 4, "bf16": 2, "e4m3": 1}
+# Weight formats in the workload line. Both block-scaled tensor-core paths
+# (e4m3 tokens against e4m3 or MX FP4 weights) are rated at the 8-bit peak,
+# twice the measured bf16 one.
+WEIGHT_DESC = {"e4m3": "e4m3 128x128-block weights, bf16 tokens",
+               "e2m1": "MX FP4 weights (e2m1, UE8M0 per 32), e4m3 tokens, bf16 x"}
 
 
 def route_bytes(spec):
@@ -429,7 +434,8 @@ def run_report(args):
     hbm = peaks["hbm_gbs"]
     cases = [W.spec("tiny"), W.spec("decode"), W.spec("prefill"), W.spec("skew"),
              W.spec("decode", shared=1), W.spec("prefill", shared=1),
-             W.spec("prefill", compact=1), W.spec("skew", compact=1)] + \
+             W.spec("prefill", compact=1), W.spec("skew", compact=1),
+             W.spec("decode_fp4"), W.spec("prefill_fp4")] + \
         [W.spec("sweep", T=t) for t in W.SWEEP_T]
     for spec in cases:
         inp = W.make_inputs(spec, seed=args.seed, device=dev)
@@ -467,7 +473,7 @@ def run_report(args):
         else:
             abytes, touched = ffn_algorithmic_bytes(spec, counts)
             flops = ffn_flops(spec, int(counts.sum()))
-            tc_peak = peaks["bf16_tflops"] * (2.0 if spec.weight == "e4m3" else 1.0)
+            tc_peak = peaks["bf16_tflops"] * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0)
             line["ffn_GBps"] = abytes / (st[2] / 1e3) / 1e9
             line["ffn_TFLOPs"] = flops / (st[2] / 1e3) / 1e12
             line["ffn_frac_hbm"] = line["ffn_GBps"] / hbm
@@ -602,12 +608,12 @@ def run_ours(args):
         # decode-size GEMMs stream weights (HBM bound); big-batch GEMMs are
         # bound by the tensor pipe
         t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
-        t_tc = flops / (peaks["bf16_tflops"] * 1e12 * (2.0 if spec.weight == "e4m3" else 1.0))
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12 * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0))
         if t_hbm >= t_tc:
             roofline = {"bound": "hbm", "achieved": bw, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": bw / peaks["hbm_gbs"]}
         else:
-            pk = peaks["bf16_tflops"] * (2.0 if spec.weight == "e4m3" else 1.0)
+            pk = peaks["bf16_tflops"] * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0)
             ach = flops / (ffn_ms / 1000.0) / 1e12
             roofline = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
                         "frac": ach / pk}
@@ -636,7 +642,7 @@ def run_ours(args):
             "data": "synthetic (seeded; random-init weights, no checkpoint)",
             "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
                                    f"top-{spec.k}{' + 1 shared expert' if spec.shared else ''} I={spec.I} "
-                                   f"{'e4m3 128x128-block weights, bf16 tokens' if spec.weight == 'e4m3' else spec.weight}",
+                                   f"{WEIGHT_DESC.get(spec.weight, spec.weight)}",
                        "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I, "shared_experts": spec.shared,
                        "compact_windows": spec.compact,
                        "parallelism": f"replicas x{world}",

@@ -245,7 +245,7 @@ cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_
   Args a;
   a.xq = b.xq; a.xs = b.xs; a.hq = b.hq; a.hs = b.hs; a.y = y;
   a.wg = w.w_gate; a.wu = w.w_up; a.wd = w.w_down;
-  a.sg = w.s_gate; a.su = w.s_up; a.sd = w.s_down;
+  a.sg = (const float*)w.s_gate; a.su = (const float*)w.s_up; a.sd = (const float*)w.s_down;
   a.H = (int)c.s.H; a.I = (int)c.s.I; a.E = (int)c.s.E;
   a.tiles = c.L.tiles;
   a.xq_dt = c.s.xq_dtype; a.w_dt = c.s.weight_dtype; a.h_dt = c.s.h_dtype; a.y_dt = c.s.y_dtype;

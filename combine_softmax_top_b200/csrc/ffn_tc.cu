@@ -77,6 +77,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColSfa0 = 448, kColSfa1 = 452, kColSfb0 = 456;
 
 enum : int { kKindGateUp = 0, kKindDown = 1, kKindEnd = 2, kKindAbort = 3 };
+// weight formats: bf16 (kind::f16), e4m3 with fp32 128 x 128 block scales, and
+// MX FP4 (e2m1, a UE8M0 scale per 32 along K) against e4m3 tokens, both
+// kind::mxf8f6f4.block_scale
+enum : int { kWBf16 = 0, kWE4m3 = 1, kWE2m1 = 2 };
 // counter-set misc slots used here: FFN calls completed on this dispatch, CTAs
 // that left the current call, the next unit to hand out
 enum : int { kFfnGen = 3, kFfnExit = 4, kFfnNext = 5 };
@@ -84,9 +88,9 @@ enum : int { kFfnGen = 3, kFfnExit = 4, kFfnNext = 5 };
 struct TcParams {
   CUtensorMap tm_wg, tm_wu, tm_wd;
   CUtensorMap tm_x[4], tm_h[4];   // token rows in boxes of 16, 32, 64, 128 rows
-  const float* sg;
-  const float* su;
-  const float* sd;
+  const void* sg;   // weight scales: fp32 per 128 x 128 block (e4m3) or UE8M0 atoms (e2m1)
+  const void* su;
+  const void* sd;
   void* hq;
   float* hs;
   void* y;
@@ -199,8 +203,10 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.f + expf
 // UE8M0 code of a power-of-two fp32 scale: its biased exponent.
 __device__ __forceinline__ uint32_t ue8m0(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
-template <bool kFp8, int kBRows>
+template <int kW, int kBRows>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr bool kFp8 = kW != kWBf16;   // block-scaled MMA, e4m3 tokens
+  constexpr bool kW4 = kW == kWE2m1;    // 4-bit weights
   using S = Stage<kBRows>;
   constexpr int kStages = S::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -433,17 +439,31 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const int brow = j.slot * kTileRows + j.row_off;
       const int64_t tile_g = j.slot;
       const bool dual = !down || j.pair;   // two weight tiles share the token tile
-      const uint32_t tx = (dual ? 2u : (uint32_t)j.nslab) * kABytes + (uint32_t)(j.nslab * N * kSlab);
+      // a weight tile lands as 128 x 128 bytes; 4-bit weights travel as half
+      // that (the copy spreads each 8 bytes of codes over 16 in shared memory)
+      constexpr uint32_t kABytesIn = kW4 ? kABytes / 2 : kABytes;
+      const uint32_t na = dual ? 2u : (uint32_t)j.nslab;   // weight tiles (and 4-bit scale atoms) per stage
+      const uint32_t tx = na * kABytesIn + (uint32_t)(j.nslab * N * kSlab);
       // the job's weight scales, one per 128 x 128 block along K: lane l holds
       // the exponents of blocks l and l + 32 (gate/down in sa, up in sb), read
       // once per job
       uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
       int sbase = 0;   // first K block held in sa*/sb*
       const int nkb = down ? p.I / 128 : p.H / 128;
-      const float* pa = down ? p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * nkb
-                             : p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
-      const float* pb = down ? p.sd + ((int64_t)j.e * p.n_hslices + j.slice + 1) * nkb
-                             : p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      const float* pa = down ? (const float*)p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * nkb
+                             : (const float*)p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      const float* pb = down ? (const float*)p.sd + ((int64_t)j.e * p.n_hslices + j.slice + 1) * nkb
+                             : (const float*)p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      // 4-bit weights: the scale atoms of the job's weight tiles, one per
+      // 128-value K block (row-major over [slice][K block])
+      const uint8_t* atom_a = nullptr;
+      const uint8_t* atom_b = nullptr;
+      if constexpr (kW4) {
+        const int n_out = down ? p.n_hslices : p.n_islices;
+        atom_a = (const uint8_t*)(down ? p.sd : p.sg) + ((int64_t)j.e * n_out + j.slice) * nkb * kSfAtomBytes;
+        atom_b = down ? atom_a + (int64_t)nkb * kSfAtomBytes
+                      : (const uint8_t*)p.su + ((int64_t)j.e * n_out + j.slice) * nkb * kSfAtomBytes;
+      }
       auto load_scales = [&](int base) {
         if (lane + base < nkb) sa0 = ue8m0(__ldg(pa + base + lane));
         if (lane + base + 32 < nkb) sa1 = ue8m0(__ldg(pa + base + lane + 32));
@@ -463,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         }
         return w;
       };
-      if constexpr (kFp8) load_scales(0);
+      if constexpr (kW == kWE4m3) load_scales(0);
       bool ok = true;
       for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         // scale atoms cover four K blocks: they travel with the stage that
         // starts a group of four
         const bool sf_stage = kFp8 && (kb0 & 3) == 0;
-        if constexpr (kFp8) {
+        if constexpr (kW == kWE4m3) {
           if (sf_stage) {
             // weight scale atoms: one exponent per 128 x 128 block, the same
             // for all 128 rows; byte b = block kb0 + b
@@ -500,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         // chosen at run time costs about four times as much to issue.
         if (ptx::elect_one()) {
           uint64_t* fb = full + stage;
-          ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (j.wide ? 2u : 1u) * (uint32_t)kSfAtomBytes : 0u));
+          ptx::mbar_arrive_expect_tx(fb, tx + (sf_stage ? (j.wide ? 2u : 1u) * (uint32_t)kSfAtomBytes : 0u) +
+                                             (kW4 ? na * (uint32_t)kSfAtomBytes : 0u));
           const int kx0 = kb0 * p.kelems;
           if (down) {
             if constexpr (kBRows <= 64) {
@@ -559,6 +580,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               ptx::bulk_load(st + S::kOffSfb1, sfb + ((tile_g + 1) * groups + kb0 / 4) * kSfAtomBytes, kSfAtomBytes,
                              fb);
           }
+          if constexpr (kW4) {   // the weight tiles' scale atoms of this stage
+            if (dual) {
+              ptx::bulk_load(st + S::kOffSfa0, atom_a + (int64_t)kb0 * kSfAtomBytes, kSfAtomBytes, fb);
+              ptx::bulk_load(st + S::kOffSfa1, atom_b + (int64_t)kb0 * kSfAtomBytes, kSfAtomBytes, fb);
+            } else {
+              for (int s = 0; s < j.nslab; ++s)
+                ptx::bulk_load(st + (s ? S::kOffSfa1 : S::kOffSfa0), atom_a + (int64_t)(kb0 + s) * kSfAtomBytes,
+                               kSfAtomBytes, fb);
+            }
+          }
         }
         __syncwarp();
         armed |= 1u << stage;
@@ -613,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       ptx::tc_fence_after();
       const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
-      const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0) : ptx::idesc_bf16(128, N);
+      const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0, kW4 ? ptx::kMxE2M1 : ptx::kMxE4M3)
+                                  : ptx::idesc_bf16(128, N);
       // the token scale atom covers the whole 128-row tile (row m in TMEM
       // column m / 32); a chunk starting at row_off reads from column row_off / 32
       const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
@@ -632,23 +664,33 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         auto sfid = [](int kb) -> uint32_t { return (uint32_t)(kb & 3); };
         if (ptx::elect_one()) {
           if constexpr (kFp8) {
-            if ((kb0 & 3) == 0) {   // a new group of four K blocks: its scale atoms
-              // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
-              ptx::tmem_cp_32x128b_x4(tmem + kColSfa0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa0), 16, 128, ptx::kLayoutNone));
-              ptx::tmem_cp_32x128b_x4(tmem + kColSfb0, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb0), 16, 128, ptx::kLayoutNone));
-              if (j.wide)   // the joined tail's rows 128.. read columns kColSfb0 + 4 ..
-                ptx::tmem_cp_32x128b_x4(tmem + kColSfb0 + 4, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfb1), 16, 128, ptx::kLayoutNone));
-              if (dual)
-                ptx::tmem_cp_32x128b_x4(tmem + kColSfa1, ptx::smem_desc(ptx::smem_u32(st + S::kOffSfa1), 16, 128, ptx::kLayoutNone));
+            // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
+            auto sf_cp = [&](uint32_t col, int off) {
+              ptx::tmem_cp_32x128b_x4(tmem + col, ptx::smem_desc(ptx::smem_u32(st + off), 16, 128, ptx::kLayoutNone));
+            };
+            if ((kb0 & 3) == 0) {   // a new group of four K blocks: the tokens' scale atoms
+              sf_cp(kColSfb0, S::kOffSfb0);
+              if (j.wide) sf_cp(kColSfb0 + 4, S::kOffSfb1);   // the joined tail's rows 128.. read columns kColSfb0 + 4 ..
+              if constexpr (kW == kWE4m3) {                   // and the weights' (one exponent per block)
+                sf_cp(kColSfa0, S::kOffSfa0);
+                if (dual) sf_cp(kColSfa1, S::kOffSfa1);
+              }
+            }
+            if constexpr (kW4) {   // 4-bit weights: new scale atoms every K block
+              sf_cp(kColSfa0, S::kOffSfa0);
+              if (dual || j.nslab == 2) sf_cp(kColSfa1, S::kOffSfa1);
             }
           }
+          // The weights' scale byte: the K block's (e4m3, one exponent per
+          // 128 x 128 block) or, for 4-bit weights, the 32-value group's.
           if (dual) {
             const uint32_t id = sfid(kb0);
-            const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
-            const uint32_t sa0 = (tmem + kColSfa0) | (id << 30), sa1 = (tmem + kColSfa1) | (id << 30);
             const uint32_t sb = (tmem + kColSfb0 + sfb_off) | (id << 30);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t ida = kW4 ? (uint32_t)kk : id;
+              const uint32_t idesc_k = idesc | (id << 4) | (ida << 29);
+              const uint32_t sa0 = (tmem + kColSfa0) | (ida << 30), sa1 = (tmem + kColSfa1) | (ida << 30);
               const uint32_t acc = (st_i > 0 || kk > 0) ? 1u : 0u;
               const uint64_t off = (uint64_t)(kk * 32) >> 4;   // 32 bytes of K per MMA
               if constexpr (kFp8) {
@@ -664,11 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               const uint64_t as = sl ? a1 : a0;
               const uint64_t bs = ptx::desc_kmajor_sw128(st + S::kOffB + sl * N * kSlab);
               const uint32_t id = sfid(kb0 + sl);
-              const uint32_t idesc_k = idesc | (id << 4) | (id << 29);
-              const uint32_t sa = (tmem + kColSfa0) | (id << 30);
               const uint32_t sb = (tmem + kColSfb0 + sfb_off) | (id << 30);
+              const uint32_t col_sa = (kW4 && sl) ? kColSfa1 : kColSfa0;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t ida = kW4 ? (uint32_t)kk : id;
+                const uint32_t idesc_k = idesc | (id << 4) | (ida << 29);
+                const uint32_t sa = (tmem + col_sa) | (ida << 30);
                 const uint32_t acc = (st_i > 0 || sl > 0 || kk > 0) ? 1u : 0u;
                 const uint64_t off = (uint64_t)(kk * 32) >> 4;
                 if constexpr (kFp8) {
@@ -902,44 +946,55 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D row-major [rows, cols] tensor, boxes of (box_cols x box_rows), 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int64_t cols, int64_t rows, int box_cols,
+// Element kinds of a tensor map: bf16, bytes (e4m3), and packed 4-bit codes
+// that land 16 codes per 16 bytes in shared memory (8 bytes of codes, 8 of
+// gap), the layout the block-scaled MMA reads 4-bit operands from.
+enum TmapElem { kElBf16, kElU8, kElU4Spread };
+
+// 2-D row-major [rows, cols] tensor (cols in elements), boxes of
+// (box_cols x box_rows), 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, TmapElem el, int64_t cols, int64_t rows, int box_cols,
                int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const int elem = fp8 ? 1 : 2;
+  const int64_t row_bytes = el == kElBf16 ? cols * 2 : (el == kElU8 ? cols : cols / 2);
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(cols * elem)};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUtensorMapDataType dt = el == kElBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : (el == kElU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B);
+  CUresult r = fn(m, dt, 2,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <bool kFp8, int kBRows>
+template <int kW, int kBRows>
 cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
   using S = Stage<kBRows>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(ffn_tc_kernel<kFp8, kBRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(ffn_tc_kernel<kW, kBRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     S::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   TcParams p;
   memset(&p, 0, sizeof(p));
   const int64_t H = c.s.H, I = c.s.I, E = c.s.E, rows = c.L.tiles * kTileRows;
-  const int kel = kFp8 ? 128 : 64;
-  if (!make_tmap(&p.tm_wg, w.w_gate, kFp8, H, E * I, kel, 128) ||
-      !make_tmap(&p.tm_wu, w.w_up, kFp8, H, E * I, kel, 128) ||
-      !make_tmap(&p.tm_wd, w.w_down, kFp8, I, E * H, kel, 128))
+  constexpr bool kFp8 = kW != kWBf16;
+  const int kel = kFp8 ? 128 : 64;   // elements per 128-byte slab row in shared memory
+  const TmapElem wel = kW == kWE2m1 ? kElU4Spread : (kFp8 ? kElU8 : kElBf16);
+  const TmapElem tel = kFp8 ? kElU8 : kElBf16;
+  if (!make_tmap(&p.tm_wg, w.w_gate, wel, H, E * I, kel, 128) ||
+      !make_tmap(&p.tm_wu, w.w_up, wel, H, E * I, kel, 128) ||
+      !make_tmap(&p.tm_wd, w.w_down, wel, I, E * H, kel, 128))
     return cudaErrorInvalidValue;
   for (int bx = 0; bx < 4; ++bx) {
-    if (!make_tmap(&p.tm_x[bx], b.xq, kFp8, H, rows, kel, 16 << bx) ||
-        !make_tmap(&p.tm_h[bx], b.hq, kFp8, I, rows, kel, 16 << bx))
+    if (!make_tmap(&p.tm_x[bx], b.xq, tel, H, rows, kel, 16 << bx) ||
+        !make_tmap(&p.tm_h[bx], b.hq, tel, I, rows, kel, 16 << bx))
       return cudaErrorInvalidValue;
   }
   p.sg = w.s_gate;
@@ -963,7 +1018,7 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.hgroups = (int)c.L.hgroups;
   p.igroups = (int)c.L.igroups;
   p.tiles = c.L.tiles;
-  ffn_tc_kernel<kFp8, kBRows><<<c.num_sms, kThreads, S::kSmemBytes, c.stream>>>(p);
+  ffn_tc_kernel<kW, kBRows><<<c.num_sms, kThreads, S::kSmemBytes, c.stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -971,11 +1026,11 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
 // they suit layers whose experts see few tokens each (decode). Bigger tiles are
 // split into 64-row chunks, which re-streams their weights, so layers with
 // many tokens per expert use 128-row tiles.
-template <bool kFp8>
+template <int kW>
 cudaError_t launch_by_rows(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
   const int64_t rows_per_expert = c.s.T * c.s.topk / c.s.E;
-  if (rows_per_expert <= 32) return launch_typed<kFp8, 64>(c, b, w, y);
-  return launch_typed<kFp8, 128>(c, b, w, y);
+  if (rows_per_expert <= 32) return launch_typed<kW, 64>(c, b, w, y);
+  return launch_typed<kW, 128>(c, b, w, y);
 }
 
 }  // namespace
@@ -984,13 +1039,14 @@ bool ffn_tc_supported(const moe_shape& s) {
   if (s.identity_experts) return false;
   const bool bf16 = s.xq_dtype == MOE_BF16 && s.weight_dtype == MOE_BF16 && s.h_dtype == MOE_BF16 &&
                     s.y_dtype == MOE_BF16;
-  const bool fp8 = s.xq_dtype == MOE_E4M3 && s.weight_dtype == MOE_E4M3 && s.h_dtype == MOE_E4M3 &&
-                   s.y_dtype == MOE_BF16;
+  const bool fp8 = s.xq_dtype == MOE_E4M3 && (s.weight_dtype == MOE_E4M3 || s.weight_dtype == MOE_E2M1) &&
+                   s.h_dtype == MOE_E4M3 && s.y_dtype == MOE_BF16;
   return (bf16 || fp8) && s.H % 128 == 0 && s.I % 128 == 0;
 }
 
 cudaError_t launch_ffn_tc(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
-  return c.s.weight_dtype == MOE_E4M3 ? launch_by_rows<true>(c, b, w, y) : launch_by_rows<false>(c, b, w, y);
+  if (c.s.weight_dtype == MOE_E2M1) return launch_by_rows<kWE2m1>(c, b, w, y);
+  return c.s.weight_dtype == MOE_E4M3 ? launch_by_rows<kWE4m3>(c, b, w, y) : launch_by_rows<kWBf16>(c, b, w, y);
 }
 
 }  // namespace moe

@@ -10,6 +10,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 namespace {
 
+// activation, row and output dtypes (E2M1 is a weight dtype only)
 bool is_dtype(int32_t d) { return d == MOE_F32 || d == MOE_BF16 || d == MOE_E4M3; }
 
 }  // namespace
@@ -46,7 +47,8 @@ moe_status check_shape(const moe_shape* s) {
   }
   if (s->identity_experts) return MOE_OK;
   if (s->I <= 0 || s->I > (1 << 24) || s->I % 16 != 0) return MOE_ERR_INVALID_ARG;
-  if (!is_dtype(s->weight_dtype) || !is_dtype(s->h_dtype) || !is_dtype(s->y_dtype))
+  if ((!is_dtype(s->weight_dtype) && s->weight_dtype != MOE_E2M1) || !is_dtype(s->h_dtype) ||
+      !is_dtype(s->y_dtype))
     return MOE_ERR_INVALID_ARG;
   if (s->y_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   const bool f32 = s->act_dtype == MOE_F32 && s->xq_dtype == MOE_F32 && s->weight_dtype == MOE_F32 &&
@@ -57,7 +59,11 @@ moe_status check_shape(const moe_shape* s) {
   const bool fp8 = s->act_dtype == MOE_BF16 && s->xq_dtype == MOE_E4M3 &&
                    s->weight_dtype == MOE_E4M3 && s->h_dtype == MOE_E4M3 &&
                    s->y_dtype == MOE_BF16 && s->out_dtype == MOE_BF16;
-  if (!f32 && !bf16 && !fp8) return MOE_ERR_UNSUPPORTED;
+  // MX FP4 weights with e4m3 tokens (block-scaled MMA of mixed operand types)
+  const bool fp4w = s->act_dtype == MOE_BF16 && s->xq_dtype == MOE_E4M3 &&
+                    s->weight_dtype == MOE_E2M1 && s->h_dtype == MOE_E4M3 &&
+                    s->y_dtype == MOE_BF16 && s->out_dtype == MOE_BF16;
+  if (!f32 && !bf16 && !fp8 && !fp4w) return MOE_ERR_UNSUPPORTED;
   // the expert FFN kernels work on 128-feature slices
   if (s->H % kQBlock != 0 || s->I % kQBlock != 0) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -106,6 +112,14 @@ moe_status check_weights(const moe_shape* s, const moe_weights* w) {
   if (!w || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
   if (s->weight_dtype == MOE_E4M3 && (!w->s_gate || !w->s_up || !w->s_down)) return MOE_ERR_INVALID_ARG;
+  if (s->weight_dtype == MOE_E2M1) {
+    // packed 4-bit rows are copied by the tensor-memory-access unit, which
+    // wants 32-byte aligned bases for them; scale atoms move in 16-byte units
+    auto a32 = [](const void* p) { return ((uintptr_t)p & 31u) == 0; };
+    if (!w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
+    if (!a32(w->w_gate) || !a32(w->w_up) || !a32(w->w_down)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->s_gate) || !aligned16(w->s_up) || !aligned16(w->s_down)) return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 

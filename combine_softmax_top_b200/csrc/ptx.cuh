@@ -238,10 +238,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
-// Instruction descriptor, kind::mxf8f6f4 block-scaled, e4m3 A/B, UE8M0 scales.
-__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) {
+// Operand formats of kind::mxf8f6f4.
+constexpr uint32_t kMxE4M3 = 0, kMxE2M1 = 5;
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled, A in a_fmt (e4m3 or
+// e2m1), B e4m3, UE8M0 scales.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id, uint32_t a_fmt = kMxE4M3) {
   return ((sf_id & 3) << 4)            // B scale-factor id
-         | (0u << 7) | (0u << 10)      // A, B format: e4m3
+         | (a_fmt << 7) | (kMxE4M3 << 10)   // A, B format
          | ((uint32_t)(N >> 3) << 17)
          | (1u << 23)                  // scale format: UE8M0
          | ((uint32_t)(M >> 4) << 24)

@@ -12,13 +12,13 @@ from dataclasses import dataclass
 
 import torch
 
-from .workloads import BF16, E4M3, F32, Spec
+from .workloads import BF16, E2M1, E4M3, F32, Spec
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
-MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
-_DT = {F32: MOE_F32, BF16: MOE_BF16, E4M3: MOE_E4M3}
+MOE_F32, MOE_BF16, MOE_E4M3, MOE_E2M1 = 0, 1, 2, 3
+_DT = {F32: MOE_F32, BF16: MOE_BF16, E4M3: MOE_E4M3, E2M1: MOE_E2M1}
 _TORCH = {F32: torch.float32, BF16: torch.bfloat16, E4M3: torch.uint8}
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
@@ -260,9 +260,10 @@ def run_layer(b: Buffers, inp: dict, stream=None) -> None:
 
 
 # kernels the library launches per stage (mirrors the launch plan in csrc/)
-_FFN_KERNELS = {F32: 2, BF16: 1, E4M3: 1}
+_FFN_KERNELS = {F32: 2, BF16: 1, E4M3: 1, E2M1: 1}
 
 
 def kernels_per_layer(s: Spec) -> int:
-    """route + dispatch + grouped FFN + combine launches of one moe_layer."""
-    return 3 + (0 if s.identity else _FFN_KERNELS[s.weight])
+    """route + dispatch (+ its counting pass with compact windows) + grouped
+    FFN + combine launches of one moe_layer."""
+    return 3 + (1 if s.compact else 0) + (0 if s.identity else _FFN_KERNELS[s.weight])

@@ -59,7 +59,8 @@ typedef struct CUstream_st* moe_stream_t;
 typedef enum moe_dtype {
   MOE_F32 = 0,   /* IEEE binary32 */
   MOE_BF16 = 1,  /* bfloat16 */
-  MOE_E4M3 = 2   /* OCP FP8 E4M3 with power-of-two fp32 block scales */
+  MOE_E4M3 = 2,  /* OCP FP8 E4M3 with power-of-two fp32 block scales */
+  MOE_E2M1 = 3   /* OCP MX FP4 E2M1, two per byte, UE8M0 scale per 32 (weights only) */
 } moe_dtype;
 
 typedef enum moe_status {
@@ -80,6 +81,9 @@ typedef enum moe_status {
  *   fp32 layer      F32,  F32,  F32,  F32,  F32,  F32
  *   bf16 layer      BF16, BF16, BF16, BF16, BF16, BF16
  *   fp8 layer       BF16, E4M3, E4M3, E4M3, BF16, BF16
+ *   fp4-weight layer BF16, E4M3, E2M1, E4M3, BF16, BF16 (MX FP4 weights: the
+ *                   GC-MoE explainer's "Two MMA Implementations" names 4-bit
+ *                   weights whose 32-element blocks share one exponent)
  *   identity experts (identity_experts = 1): act BF16/F32, xq any, out BF16/F32;
  *                   weight/h/y ignored, moe_grouped_ffn is a no-op.
  * H must be a multiple of 16 (of quant_block = 128 when xq is E4M3); with
@@ -167,16 +171,24 @@ typedef struct moe_dispatch_bufs {
  *   w_gate, w_up [E, I, H]; w_down [E, H, I], in weight_dtype.
  *   E4M3 weights carry one fp32 scale per 128 x 128 block:
  *   s_gate, s_up [E, I/128, H/128]; s_down [E, H/128, I/128]. Scales must be
- *   powers of two (the tensor cores apply them as 8-bit exponents). NULL for
- *   other weight dtypes.
+ *   powers of two (the tensor cores apply them as 8-bit exponents).
+ *   E2M1 weights hold two 4-bit codes per byte, element 2i of a row in the
+ *   low nibble of its byte i (w_gate, w_up [E, I, H/2] bytes; w_down
+ *   [E, H, I/2]; each matrix 32-byte aligned), and one UE8M0 scale byte
+ *   (value 2^(byte - 127), byte < 255) per 32 consecutive elements of a row,
+ *   stored in the tensor cores' scale-atom order: s_gate, s_up
+ *   [E, I/128, H/128, 512] bytes, s_down [E, H/128, I/128, 512]; inside the
+ *   atom of a 128 x 128 block, row r's scale of elements 32 b .. 32 b + 31 of
+ *   the block (b = 0..3) is byte (r % 32) * 16 + (r / 32) * 4 + b.
+ *   NULL for unscaled weight dtypes.
  */
 typedef struct moe_weights {
   const void* w_gate;
   const void* w_up;
   const void* w_down;
-  const float* s_gate;
-  const float* s_up;
-  const float* s_down;
+  const void* s_gate;
+  const void* s_up;
+  const void* s_down;
 } moe_weights;
 
 /* Workspace size in bytes for `shape` (host only, enqueues nothing). */

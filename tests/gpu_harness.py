@@ -10,7 +10,7 @@ from combine_softmax_top_b200 import moe
 from combine_softmax_top_b200 import workloads as W
 from tests.helpers import raw
 
-ODT = {W.F32: oracle.F32, W.BF16: oracle.BF16, W.E4M3: oracle.E4M3}
+ODT = {W.F32: oracle.F32, W.BF16: oracle.BF16, W.E4M3: oracle.E4M3, W.E2M1: oracle.E2M1}
 
 
 def run_stages(s: W.Spec, inp: dict, layer: bool = False) -> moe.Buffers:
@@ -43,7 +43,8 @@ def oracle_problem(s: W.Spec, inp: dict, experts=None) -> oracle.Problem:
     if not s.identity:
         es = range(s.ne) if experts is None else sorted(set(int(e) for e in experts) | ({s.E} if s.shared else set()))
         for name in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
-            t = inp.get(name)
+            # 4-bit weights: the oracle reads the per-row scales, the library the atoms
+            t = inp.get(name + "_rows" if (s.weight == W.E2M1 and name[0] == "s") else name)
             if t is not None:
                 kw[name] = {e: raw(t[e]) for e in es}
     return oracle.Problem(s.T, s.H, s.E, s.k, s.I, **kw)

@@ -130,3 +130,15 @@ def test_noalloc_dispatch_refuses_compact_windows():
     compact flag is refused before any pointer is looked at."""
     sh = moe.make_shape(W.spec("decode", compact=1))
     assert moe.lib().moe_dispatch_noalloc(ctypes.byref(sh), None, None, None, None) == 2
+
+
+def test_fp4_weight_layer_shape_accepted_and_e2m1_only_for_weights():
+    """MX FP4 (E2M1) is a weight dtype: the fp4-weight layer (bf16 x, e4m3
+    tokens and h, E2M1 weights) is accepted; E2M1 anywhere else is refused."""
+    sh = moe.make_shape(W.spec("decode_fp4"))
+    n = ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_bytes(ctypes.byref(sh), ctypes.byref(n)) == 0 and n.value > 0
+    for field in ("act_dtype", "xq_dtype", "h_dtype", "y_dtype", "out_dtype"):
+        bad = moe.make_shape(W.spec("decode_fp4"))
+        setattr(bad, field, moe.MOE_E2M1)
+        assert moe.lib().moe_workspace_bytes(ctypes.byref(bad), ctypes.byref(n)) in (1, 2), field
