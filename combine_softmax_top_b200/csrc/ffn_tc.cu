@@ -219,11 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   uint64_t* drain = acc_empty + 2;
   uint64_t* uq_full = drain + 1;              // [kUQ] job queue
   uint64_t* uq_empty = uq_full + kUQ;         // [kUQ]
-  static_assert((2 * kStages + 5 + 2 * kUQ) * 8 <= 256, "barriers fit before the job queue");
-  int4* uq = reinterpret_cast<int4*>(ctl + 256);               // [kUQ] packed jobs
-  int4* epi_job = reinterpret_cast<int4*>(ctl + 384);          // job broadcast to the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 400);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 404);
+  static_assert((2 * kStages + 5 + 2 * kUQ) * 8 <= 320, "barriers fit before the job queue");
+  int4* uq = reinterpret_cast<int4*>(ctl + 320);               // [kUQ] packed jobs
+  int4* epi_job = reinterpret_cast<int4*>(ctl + 448);          // job broadcast to the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 464);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 468);
   float* red = reinterpret_cast<float*>(ctl + 512);            // [2 sets][4 warps][32 tokens]
   float* sinv = reinterpret_cast<float*>(ctl + 1536);          // [2 sets][32 tokens] 1 / scale
 
@@ -264,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   uint32_t* hdone = set_hdone(set, p.E, p.tiles);
   // down units cover two slices of H each when tiles are large (the two share
   // the token tile, like gate and up)
-  const int dpair = (kBRows > 64 && (p.n_hslices & 1) == 0) ? 2 : 1;
+  // (and with the 16-row variant, whose stage has room for one token slab
+  // only: a pair keeps two weight tiles in every stage)
+  const int dpair = ((kBRows > 64 || kBRows <= 16) && (p.n_hslices & 1) == 0) ? 2 : 1;
   Header* hdr = p.ws.hdr;
 
   // Take job i from the queue (one lane of a consumer role).
@@ -527,9 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
                                              (kW4 ? na * (uint32_t)kSfAtomBytes : 0u));
           const int kx0 = kb0 * p.kelems;
           if (down) {
-            if constexpr (kBRows <= 64) {
-              for (int s = 0; s < j.nslab; ++s)
-                ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow, pol);
+            if constexpr (kBRows <= 64) {   // one slab of slices (slice, slice + 1), or nslab slabs of one slice
+              if (j.pair) {
+                ptx::tma_load_2d_hint(st, &p.tm_wd, fb, kx0, arow, pol);
+                ptx::tma_load_2d_hint(st + S::kOffA1, &p.tm_wd, fb, kx0, arow + 128, pol);
+              } else {
+                for (int s = 0; s < j.nslab; ++s)
+                  ptx::tma_load_2d_hint(st + s * S::kOffA1, &p.tm_wd, fb, kx0 + s * p.kelems, arow, pol);
+              }
             } else {   // one slab of slices (slice, slice + 1), or nslab slabs of one slice
               if (j.pair) {
                 ptx::tma_load_2d(st, &p.tm_wd, fb, kx0, arow);
@@ -650,8 +657,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const uint32_t idesc = kFp8 ? ptx::idesc_mxf8(128, N, 0, kW4 ? ptx::kMxE2M1 : ptx::kMxE4M3)
                                   : ptx::idesc_bf16(128, N);
       // the token scale atom covers the whole 128-row tile (row m in TMEM
-      // column m / 32); a chunk starting at row_off reads from column row_off / 32
-      const uint32_t sfb_off = (uint32_t)j.row_off / 32u;
+      // column m / 32, lane m % 32); a chunk starting at row_off (a multiple
+      // of 64 with 64-row chunks) reads from column row_off / 32. A 16-row
+      // chunk inside a tile gets its rows gathered into lanes 0-15 of a
+      // scratch atom's first column instead (below).
+      const bool sfb_gather = kFp8 && kBRows <= 16 && j.row_off != 0;
+      const uint32_t sfb_off = kBRows <= 16 ? 0u : (uint32_t)j.row_off / 32u;
       for (int st_i = 0; st_i < nsteps; ++st_i) {
         int w_ok = 1;
         if (lane == 0) w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x60000000u | stage);
@@ -665,6 +676,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         // scale-factor byte of a K block inside its atom: in the instruction
         // descriptor and in the top two bits of the scale addresses
         auto sfid = [](int kb) -> uint32_t { return (uint32_t)(kb & 3); };
+        if (sfb_gather && (kb0 & 3) == 0) {   // into the SFB1 slot, which 16-row stages leave unused
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(st + S::kOffSfb0);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(st + S::kOffSfb1);
+          if (lane < 16) {
+            const int m = j.row_off + lane;   // < 128: row_off <= 112
+            dst[lane * 4] = src[(m % 32) * 4 + m / 32];
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+        }
         if (ptx::elect_one()) {
           if constexpr (kFp8) {
             // 32 rows x 16 bytes, no swizzle: 8-row core matrices 128 bytes apart
@@ -672,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
               ptx::tmem_cp_32x128b_x4(tmem + col, ptx::smem_desc(ptx::smem_u32(st + off), 16, 128, ptx::kLayoutNone));
             };
             if ((kb0 & 3) == 0) {   // a new group of four K blocks: the tokens' scale atoms
-              sf_cp(kColSfb0, S::kOffSfb0);
+              sf_cp(kColSfb0, sfb_gather ? S::kOffSfb1 : S::kOffSfb0);
               if (j.wide) sf_cp(kColSfb0 + 4, S::kOffSfb1);   // the joined tail's rows 128.. read columns kColSfb0 + 4 ..
               if constexpr (kW == kWE4m3) {                   // and the weights' (one exponent per block)
                 sf_cp(kColSfa0, S::kOffSfa0);
@@ -1025,13 +1046,17 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   return cudaGetLastError();
 }
 
-// Token tiles of up to 64 rows give a deeper pipeline (5 stages instead of 4);
-// they suit layers whose experts see few tokens each (decode). Bigger tiles are
-// split into 64-row chunks, which re-streams their weights, so layers with
-// many tokens per expert use 128-row tiles.
+// Token tiles of up to 64 rows give a deeper pipeline (5 stages instead of 4),
+// and of up to 16 rows 6 stages; they suit layers whose experts see few tokens
+// each (decode). Bigger tiles are split into chunks of that many rows, which
+// re-streams their weights, so layers with many tokens per expert use 128-row
+// tiles.
 template <int kW>
 cudaError_t launch_by_rows(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {
   const int64_t rows_per_expert = c.s.T * c.s.topk / c.s.E;
+  // a few tokens per expert (decode): 16-row stages, six of them in flight;
+  // not with a shared expert, whose window holds all T tokens
+  if (rows_per_expert <= 4 && !c.shared) return launch_typed<kW, 16>(c, b, w, y);
   if (rows_per_expert <= 32) return launch_typed<kW, 64>(c, b, w, y);
   return launch_typed<kW, 128>(c, b, w, y);
 }

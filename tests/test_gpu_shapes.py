@@ -3,7 +3,9 @@ tails, a single token, no tokens, k = 1, a hidden size whose K loop crosses 64
 scale blocks, routing skewed so one expert's window spans several tiles
 (split into chunks by the tensor-core FFN), and layers with more than 32 rows
 per expert, whose tensor-core FFN uses 128-row tiles (down jobs over pairs of
-H slices when H/128 is even, single slices when it is odd)."""
+H slices when H/128 is even, single slices when it is odd), and layers with at
+most 4 rows per expert, whose FFN uses 16-row tiles (an expert with more rows
+is split into 16-row chunks)."""
 import numpy as np
 import pytest
 import torch
@@ -29,6 +31,12 @@ CASES = [
     ("big_tiles_pairs_fp8", "decode", dict(T=300, H=512, E=4, k=2, I=384), 0.0),     # H/128 even: down pairs
     ("big_tiles_odd_h_fp8", "decode", dict(T=300, H=384, E=4, k=2, I=256), 0.0),     # H/128 odd: single slices
     ("big_tiles_pairs_bf16", "skew", dict(T=260, H=256, E=4, k=2, I=256, zipf_s=0.0), 0.0),
+    # <= 4 rows per expert: 16-row token tiles, six pipeline stages, down pairs
+    ("r16_fp8", "decode", dict(T=64, H=512, E=64, k=4, I=256), 0.0),
+    ("r16_hot_expert_fp8", "decode", dict(T=64, H=512, E=64, k=4, I=256), 30.0),   # 64 rows: 4 chunks
+    ("r16_odd_h_fp8", "decode", dict(T=64, H=384, E=64, k=4, I=256), 0.0),         # no pairs: one slab
+    ("r16_hot_expert_fp4", "decode_fp4", dict(T=64, H=512, E=64, k=4, I=256), 30.0),
+    ("r16_bf16", "skew", dict(T=64, H=256, E=64, k=4, I=256, zipf_s=0.0), 0.0),
     ("tiny_no_renorm", "tiny", dict(renorm=0), 0.0),
     ("fp32_ragged", "tiny", dict(T=45, H=384, E=7, k=3, I=256), 0.0),
 ]
