@@ -12,15 +12,15 @@
 //  * Tokens go to experts according to the gating/routing result (GC-MoE
 //    explainer, same section). The routing rule itself, softmax over the router
 //    logits then top-k with optional renormalisation, is not printed on the
-//    pages; it is the reading this build takes (softmax is monotone, so the k
+//    pages; it is the reading taken here (softmax is monotone, so the k
 //    largest logits are the k largest probabilities).
 //  * The expert FFN is a gated (SwiGLU) FFN with a requantisation fused after
 //    the activation (GC-MoE feed item, "Full text"; explainer, "Two MMA
 //    Implementations in the Compute Partition"). SwiGLU is read as
 //    h = silu(x W_gate^T) * (x W_up^T), y = h W_down^T.
 //  * FP8 operands carry block scale factors (explainer, tcgen05 paragraph of
-//    "Two MMA Implementations"). The pages print a 32-element block; this build
-//    uses 128-element blocks with power-of-two fp32 scales, which the same
+//    "Two MMA Implementations"). The pages print a 32-element block; the layer
+//    here uses 128-element blocks with power-of-two fp32 scales, which the same
 //    block-scaled MMA consumes exactly.
 //  * 4-bit weights are the microscaling (MX) form the same paragraph names:
 //    every 32 consecutive elements share one exponent scale, and the weights
