@@ -176,7 +176,7 @@ def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None, thre
 
     all_cores = len(os.sched_getaffinity(0))
     cores = oracle.set_threads(threads if threads else all_cores)
-    odt = {"f32": oracle.F32, "bf16": oracle.BF16, "e4m3": oracle.E4M3}
+    odt = {"f32": oracle.F32, "bf16": oracle.BF16, "e4m3": oracle.E4M3, "e2m1": oracle.E2M1}
 
     def host(t):
         t = t.detach().cpu().contiguous()
@@ -197,8 +197,10 @@ def oracle_sample(spec, inp, seconds: float, max_tokens: int | None = None, thre
         if not spec.identity:
             experts = sorted(set(idx[done:t1].ravel().tolist()))
             for n in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
-                if inp.get(n) is not None:
-                    kw[n] = {e: host(inp[n][e]) for e in experts}
+                # 4-bit weights: the oracle reads per-row scales, the library scale atoms
+                m = n + "_rows" if (spec.weight == "e2m1" and n[0] == "s") else n
+                if inp.get(m) is not None:
+                    kw[n] = {e: host(inp[m][e]) for e in experts}
         p = oracle.Problem(spec.T, spec.H, spec.E, spec.k, spec.I, shared=spec.shared, x_dtype=odt[spec.act],
                            xq_dtype=odt[spec.xq], w_dtype=odt[spec.weight], h_dtype=odt[spec.h],
                            y_dtype=odt[spec.y], out_dtype=odt[spec.out], renorm=spec.renorm,
