@@ -60,6 +60,9 @@ LAYER_CASES = [
     ("shared_expert", "decode_fp4", dict(T=300, H=512, E=4, k=2, I=384, shared=1)),
     ("compact", "decode_fp4", dict(T=300, H=512, E=4, k=2, I=384, compact=1)),
     ("decode", "decode_fp4", {}),
+    # <= 4 rows per expert with a shared expert: 16-row tiles, the shared
+    # expert's 64 rows in four chunks (scale words gathered for rows 16..63)
+    ("r16_shared", "decode_fp4", dict(T=64, H=512, E=64, k=4, I=256, shared=1)),
 ]
 
 
