@@ -496,6 +496,7 @@ def run_report(args):
              W.spec("decode", shared=1), W.spec("prefill", shared=1),
              W.spec("prefill", compact=1), W.spec("skew", compact=1),
              W.spec("decode_fp4"), W.spec("prefill_fp4"), W.spec("decode_fp4", shared=1)] + \
+        [W.spec("decode", T=t) for t in (1, 8, 32, 512)] + \
         [W.spec("sweep", T=t) for t in W.SWEEP_T]
     for spec in cases:
         inp = W.make_inputs(spec, seed=args.seed, device=dev)
