@@ -36,6 +36,7 @@ CASES = [
     ("r16_hot_expert_fp8", "decode", dict(T=64, H=512, E=64, k=4, I=256), 30.0),   # 64 rows: 4 chunks
     ("r16_odd_h_fp8", "decode", dict(T=64, H=384, E=64, k=4, I=256), 0.0),         # no pairs: one slab
     ("r16_hot_expert_fp4", "decode_fp4", dict(T=64, H=512, E=64, k=4, I=256), 30.0),
+    ("r16_odd_h_fp4", "decode_fp4", dict(T=64, H=384, E=64, k=4, I=256), 0.0),      # one 4-bit slab per stage
     ("r16_bf16", "skew", dict(T=64, H=256, E=64, k=4, I=256, zipf_s=0.0), 0.0),
     # MX FP4 weights and compact windows off the standard shapes
     ("one_token_fp4", "decode_fp4", dict(T=1, H=512, E=16, k=4, I=256), 0.0),
