@@ -94,8 +94,9 @@ typedef enum moe_status {
  *
  * flags = MOE_FLAG_SHARED_EXPERT adds one shared expert that every token also
  * goes through, computed in the same grouped FFN launch and added to the
- * output with weight 1 (GC-MoE feed item: the compute partition fuses
- * "optionally shared experts"; the weight-1 sum is this library's reading).
+ * output with weight 1 (GC-MoE feed item: shared experts, when a model has
+ * them, are fused into the compute partition; the weight-1 sum is this
+ * library's reading).
  * E and topk stay the routed counts (logits are [T, E]); every per-expert and
  * per-pair array grows by one: the weight arrays hold E + 1 experts (the
  * shared one last, index E), topk_idx / topk_w have topk + 1 columns (moe_route
