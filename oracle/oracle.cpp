@@ -27,8 +27,8 @@
 //    shrink to 4 bits. Read as the OCP MX formats: FP4 E2M1 elements with one
 //    UE8M0 scale (2^(byte - 127)) per 32 elements along K.
 //  * Combine weights each expert output by its routing weight and sums back in
-//    token order (NVLinkOneSided abstract; Ascend report abstract, "direct
-//    reading from remote expert windows").
+//    token order (NVLinkOneSided abstract; Ascend report abstract: combine
+//    reads expert outputs straight out of the expert windows).
 //
 // Precision: every sum and product is formed in double. A value is rounded
 // only where the GPU path stores it (x to e4m3, h to fp32 then bf16/e4m3,
