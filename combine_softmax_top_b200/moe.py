@@ -26,7 +26,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 
 EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
            "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_poll_status", "moe_status_string",
-           "moe_dispatch_noalloc")
+           "moe_dispatch_noalloc", "moe_pack_mx_scales")
 
 
 class MoeError(RuntimeError):
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "moe_poll_status": [P, P],
             "moe_dispatch_noalloc": [S, P, P, ctypes.POINTER(moe_dispatch_bufs), P],
             "moe_status_string": [ctypes.c_int],
+            "moe_pack_mx_scales": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -163,6 +164,17 @@ def moe_layer(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe_disp
                                         ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
                                         ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
                                         _stream(stream)))
+
+
+def moe_pack_mx_scales(src: torch.Tensor, stream=None) -> torch.Tensor:
+    """MX FP4 weight scales [n, rows, cols/32] (uint8, device) -> the scale
+    atoms [n, rows/128, cols/128, 512] moe_weights wants (moe_pack_mx_scales)."""
+    n, rows, groups = src.shape
+    src = src.contiguous()
+    dst = torch.empty((n, rows // 128, groups * 32 // 128, 512), dtype=torch.uint8, device=src.device)
+    _check("moe_pack_mx_scales", lib().moe_pack_mx_scales(n, rows, groups * 32, _ptr(src), _ptr(dst),
+                                                           _stream(stream)))
+    return dst
 
 
 def moe_dispatch_noalloc(shape, x, topk_idx, bufs: moe_dispatch_bufs, stream=None) -> None:

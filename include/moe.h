@@ -301,6 +301,24 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x, c
                                         const moe_dispatch_bufs* bufs, moe_stream_t stream);
 
 /*
+ * Rearrange MX FP4 weight scales from row order into the scale-atom order
+ * moe_weights wants for MOE_E2M1 weights (a byte permutation on the device,
+ * no arithmetic; the GC-MoE explainer's "Two MMA Implementations" gives the
+ * 32-element shared exponent, the atom order is the tensor cores' own).
+ *   n     matrices (experts), >= 0
+ *   rows  rows of each matrix (I for gate/up, H for down), a multiple of 128
+ *   cols  elements per row (H for gate/up, I for down), a multiple of 128
+ *   src   [n, rows, cols / 32] UE8M0 bytes, device, read only
+ *   dst   [n, rows / 128, cols / 128, 512] bytes, device, written: inside the
+ *         atom of a 128 x 128 block, row r's scale of block elements
+ *         32 b .. 32 b + 31 is byte (r % 32) * 16 + (r / 32) * 4 + b
+ * src and dst must not overlap. Enqueued on `stream`; MOE_ERR_INVALID_ARG
+ * for bad sizes or NULL pointers (n * rows * cols == 0 enqueues nothing).
+ */
+MOE_API moe_status moe_pack_mx_scales(int64_t n, int64_t rows, int64_t cols, const void* src, void* dst,
+                                      moe_stream_t stream);
+
+/*
  * Synchronises `stream`, returns the first device error latched in `ws`
  * since the last poll (MOE_OK if none) and clears it.
  */

@@ -142,3 +142,13 @@ def test_fp4_weight_layer_shape_accepted_and_e2m1_only_for_weights():
         bad = moe.make_shape(W.spec("decode_fp4"))
         setattr(bad, field, moe.MOE_E2M1)
         assert moe.lib().moe_workspace_bytes(ctypes.byref(bad), ctypes.byref(n)) in (1, 2), field
+
+
+@pytest.mark.parametrize("n,rows,cols", [(1, 100, 128), (1, 128, 96), (-1, 128, 128)])
+def test_pack_mx_scales_rejects_bad_sizes(n, rows, cols):
+    """Sizes are checked on the host, before any pointer is used."""
+    assert moe.lib().moe_pack_mx_scales(n, rows, cols, None, None, None) == 1
+
+
+def test_pack_mx_scales_empty_enqueues_nothing():
+    assert moe.lib().moe_pack_mx_scales(0, 128, 128, None, None, None) == 0
