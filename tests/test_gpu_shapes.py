@@ -43,6 +43,8 @@ CASES = [
     ("ragged_fp4", "decode_fp4", dict(T=37, H=384, E=5, k=3, I=640), 0.0),
     ("one_token_compact", "decode", dict(T=1, H=512, E=16, k=4, I=256, compact=1), 0.0),
     ("hot_expert_compact_fp4", "decode_fp4", dict(T=256, H=512, E=64, k=2, I=256, compact=1), 30.0),
+    ("many_experts_compact_fp4", "decode_fp4", dict(T=64, H=256, E=1024, k=8, I=256, compact=1), 0.0),
+    ("many_experts_fp8", "decode", dict(T=64, H=256, E=1000, k=32, I=256), 0.0),
     ("tiny_no_renorm", "tiny", dict(renorm=0), 0.0),
     ("fp32_ragged", "tiny", dict(T=45, H=384, E=7, k=3, I=256), 0.0),
 ]
