@@ -379,8 +379,9 @@ def time_layer(spec, inp, b, steps, warmup, stream, flush):
 
 def time_e2e_pipelined(spec, inp, b, w, bufs, stream, flush, steps, dev):
     """Steps of H2D (x, logits) -> moe_layer -> D2H (out), copies overlapped
-    with the neighbouring steps' layers on a second stream; returns ms per
-    step from the first copy to the last."""
+    with the neighbouring steps' layers on two copy streams (one per
+    direction, so the two directions of the host link overlap too); returns
+    ms per step from the first copy to the last."""
     import torch
     from combine_softmax_top_b200 import moe
     from combine_softmax_top_b200 import workloads as W
@@ -390,7 +391,8 @@ def time_e2e_pipelined(spec, inp, b, w, bufs, stream, flush, steps, dev):
     dx = [torch.empty_like(inp["x"]) for _ in range(2)]
     dl = [torch.empty_like(inp["logits"]) for _ in range(2)]
     dout = [b.out, torch.empty_like(b.out)]
-    cs = torch.cuda.Stream(device=dev)
+    cs = torch.cuda.Stream(device=dev)        # host -> device
+    co = torch.cuda.Stream(device=dev)        # device -> host
     weight_bytes = 0 if spec.identity else W.bytes_per_expert(spec) * spec.ne
     flush_each = weight_bytes < 4 * 126 * (1 << 20)    # weights not well above the 126 MB L2
     n = steps                                      # pipeline fill and drain included (conservative)
@@ -420,17 +422,18 @@ def time_e2e_pipelined(spec, inp, b, w, bufs, stream, flush, steps, dev):
         moe.moe_layer(b.shape, dx[i % 2], dl[i % 2], w, b.topk_idx, b.topk_w, bufs, b.y, b.ws,
                       dout[i % 2], stream)
         ev_done[i].record(stream)
-        with torch.cuda.stream(cs):
-            cs.wait_event(ev_done[i])
+        with torch.cuda.stream(co):
+            co.wait_event(ev_done[i])
             ho[i % 2].copy_(dout[i % 2], non_blocking=True)
-            ev_out[i].record(cs)
+            ev_out[i].record(co)
+    cs.wait_event(ev_out[n - 1])
     t1.record(cs)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
     return {"ms": ms, "unit": "tokens/s",
             "h2d_bytes_per_step": hx.numel() * hx.element_size() + hl.numel() * hl.element_size(),
             "d2h_bytes_per_step": ho[0].numel() * ho[0].element_size(),
-            "how": "H2D of step i+1 and D2H of step i on a copy stream beside step i's layer, "
+            "how": "H2D of step i+1 and D2H of step i on two copy streams beside step i's layer, "
                    "first H2D to last D2H over all steps; "
                    + ("L2 flushed before each layer" if flush_each else "weights larger than L2, no flush")}
 
