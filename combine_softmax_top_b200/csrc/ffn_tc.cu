@@ -11,20 +11,22 @@
 // "Three-Node CUDA Graph and token-ring Handshake").
 //
 // Work units, processed in one fixed order by a persistent grid:
-//   gate/up : (ring slot, 128-feature slice of I) -> h rows of that slice
-//   down    : (ring slot, 128-feature slice of H, or two slices sharing the
-//             token tile when tiles hold up to 128 rows) -> y rows
+//   gate/up : (token tile, 128-feature slice of I) -> h rows of that slice
+//   down    : (token tile, 128-feature slice of H, or two slices sharing the
+//             token tile) -> y rows
 // All gate/up units come before all down units; a down unit waits until the
-// I/128 gate/up units of its tile have stored h (per-slot counter).
+// I/128 gate/up units of its tile have stored h (per-tile counter).
 //
 // Per CTA (352 threads): warp 10 schedules jobs; warp 0 streams K slabs of
-// 128 bytes into a 4- or 5-stage shared-memory ring with TMA, and for e4m3
-// builds the weights' UE8M0 scale atoms and bulk-copies the tokens'; warp 1
-// issues tcgen05.mma (kind::f16 for bf16, kind::mxf8f6f4.block_scale for
-// e4m3) into tensor memory; warps 2-9 read the fp32 accumulators back with
-// tcgen05.ld, apply SwiGLU and the per-128 requantisation (or round y to
-// bf16) and store. The producer and MMA warps run warp-uniform loops and one
-// elected lane issues each copy, MMA and commit. Every wait is bounded: on expiry the kernel latches
+// 128 bytes into a 4-, 5- or 6-stage shared-memory ring with TMA (token tiles
+// of up to 128, 64 or 16 rows), and for e4m3 weights builds their UE8M0 scale
+// atoms, for MX FP4 weights bulk-copies theirs, and bulk-copies the tokens';
+// warp 1 issues tcgen05.mma (kind::f16 for bf16, kind::mxf8f6f4.block_scale
+// for e4m3 or E2M1 weights against e4m3 tokens) into tensor memory; warps 2-9
+// read the fp32 accumulators back with tcgen05.ld, apply SwiGLU and the
+// per-128 requantisation (or round y to bf16) and store. The producer and MMA
+// warps run warp-uniform loops and one elected lane issues each copy, MMA and
+// commit. Every wait is bounded: on expiry the kernel latches
 // MOE_ERR_TIMEOUT, drains its copies and MMAs, frees tensor memory and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
