@@ -79,3 +79,26 @@ def test_zero_tokens(cuda_device):
     torch.cuda.synchronize()
     assert moe.moe_poll_status(b.ws) == 0
     assert b.counts.cpu().numpy().sum() == 0
+
+
+@pytest.mark.parametrize("over", [dict(), dict(compact=1), dict(weight=W.E2M1)],
+                         ids=["windows", "compact", "fp4"])
+def test_many_tokens(over, cuda_device):
+    """65 536 tokens over 8 experts (16 384 rows each, 128 tiles per window):
+    counts bit-exact, every pair placed once, and a sample of 256 tokens
+    against the oracle."""
+    s = W.spec("decode", T=65536, H=256, E=8, k=2, I=256, **over)
+    inp = W.make_inputs(s, seed=12, device="cuda")
+    b = G.run_stages(s, inp, layer=True)
+    assert G.poll(b) == 0
+    idx = b.topk_idx.cpu().numpy()
+    counts = b.counts.cpu().numpy()
+    assert np.array_equal(counts, oracle.counts(idx, s.E))
+    rows, pairs, experts = G.placed_rows(b)
+    assert np.array_equal(np.sort(pairs), np.arange(s.T * s.k))
+    t0, t1 = 30000, 30256
+    p = G.oracle_problem(s, inp)
+    r = oracle.moe_layer(p, raw(inp["x"]), raw(inp["logits"]), t0, t1)
+    assert np.array_equal(r["idx"], idx)
+    err = max_abs_rel(as_f64(raw(b.out)[t0:t1], s.out), as_f64(r["out"], s.out))
+    assert err < 2e-2, err
