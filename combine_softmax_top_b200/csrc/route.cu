@@ -7,8 +7,12 @@
 // logits go to the lower expert index, slots are in descending logit order.
 //
 // One warp per token. The row of E logits is read with coalesced 16-byte
-// loads (E % 4 == 0) into registers, k rounds of a warp-shuffle arg-max pick
-// the experts, and the softmax denominator is a warp reduction.
+// loads (E % 4 == 0) into registers. Each lane keeps the best of its own
+// logits; each of the k rounds takes the warp's best with two reductions (the
+// largest value as an order-preserving 32-bit key, then the lowest expert
+// index among the lanes holding it), and only the lane that supplied the
+// winner looks for its next best. The softmax denominator is a warp
+// reduction.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -24,6 +28,15 @@ struct Cand {
 // a beats b: larger logit, or equal logit and lower index
 __device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
   return av > bv || (av == bv && ai < bi);
+}
+
+// 32-bit key that orders like the float (no NaN; -0 already folded into +0)
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 template <int NV>  // logits per lane (multiple of 4 when VEC)
@@ -67,28 +80,36 @@ route_kernel(const float* __restrict__ logits, int T, int E, int k, int renorm, 
     return;
   }
 
+  // fold -0 into +0 so that the keys compare like the logits (-0 == +0)
+#pragma unroll
+  for (int c = 0; c < NV; ++c) v[c] += 0.f;
   unsigned taken = 0;  // bit c: element c already selected
+  float bv;            // this lane's best remaining logit and its expert
+  int bi;
+  auto local_best = [&]() {
+    bv = -INFINITY;
+    bi = INT32_MAX;
+#pragma unroll
+    for (int c = 0; c < NV; ++c)
+      if (!((taken >> c) & 1u) && beats(v[c], ix[c], bv, bi)) { bv = v[c]; bi = ix[c]; }
+  };
+  local_best();
   float sel_v = 0.f;   // lane j keeps slot j
   int sel_i = 0;
   float top = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = INT32_MAX;
+    const uint32_t key = bi == INT32_MAX ? 0u : order_key(bv);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+    const uint32_t wi = __reduce_min_sync(0xffffffffu, key == m ? (uint32_t)bi : 0xFFFFFFFFu);
+    const float wv = key_value(m);
+    if (j == 0) top = wv;
+    if (lane == j) { sel_v = wv; sel_i = (int)wi; }
+    if ((uint32_t)bi == wi) {   // the winner came from this lane
 #pragma unroll
-    for (int c = 0; c < NV; ++c) {
-      if (!((taken >> c) & 1u) && beats(v[c], ix[c], bv, bi)) { bv = v[c]; bi = ix[c]; }
+      for (int c = 0; c < NV; ++c)
+        if ((uint32_t)ix[c] == wi) taken |= 1u << c;
+      local_best();
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-    }
-#pragma unroll
-    for (int c = 0; c < NV; ++c)
-      if (ix[c] == bi) taken |= 1u << c;
-    if (j == 0) top = bv;
-    if (lane == j) { sel_v = bv; sel_i = bi; }
   }
 
   // softmax weights, max-subtracted
