@@ -117,8 +117,29 @@ def test_fp4_weight_alignment_is_checked(cuda_device):
     b = moe.alloc_buffers(s)
     w = moe.weights_struct(inp)
     w.w_gate += 16
+    w2 = moe.weights_struct(inp)
+    w2.s_up += 8                                        # scale atoms move in 16-byte units
     moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws)
     moe.moe_dispatch(b.shape, inp["x"], b.topk_idx, b.ws, b.dispatch_bufs())
-    with pytest.raises(moe.MoeError) as ei:
-        moe.moe_grouped_ffn(b.shape, b.dispatch_bufs(), w, b.ws, b.y)
-    assert ei.value.code == 1
+    for bad in (w, w2):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_grouped_ffn(b.shape, b.dispatch_bufs(), bad, b.ws, b.y)
+        assert ei.value.code == 1
+
+
+def test_fp4_compact_shared_workspace_reuse(cuda_device):
+    """4-bit weights, compact windows and a shared expert on one workspace
+    over calls with changing routing: each call gives the bits of a fresh run."""
+    s = W.spec("decode_fp4", T=96, H=512, E=32, k=4, I=256, compact=1, shared=1)
+    ins = [W.make_inputs(s, seed=sd, device="cuda") for sd in (0, 1)]
+    ins[1]["logits"][:, :3] += 50.0
+    b = moe.alloc_buffers(s)
+    outs = []
+    for i in (0, 1, 0):
+        moe.run_layer(b, ins[i])
+        torch.cuda.synchronize()
+        assert G.poll(b) == 0
+        outs.append(b.out.clone())
+    assert torch.equal(outs[0], outs[2])
+    fresh = G.run_stages(s, ins[1], layer=True)
+    assert torch.equal(fresh.out, outs[1])

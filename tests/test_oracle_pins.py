@@ -595,3 +595,27 @@ def test_e2m1_nibble_order_and_scale_index_matter():
                                 ex, xq, xs)[2]
     assert not np.array_equal(base, swapped)
     assert not np.array_equal(base, rolled)
+
+
+def test_e2m1_needs_whole_scale_groups():
+    """MX FP4 rows are made of whole 32-element scale groups: the oracle
+    refuses an H that is not a multiple of 32 (fp32 tokens, so that no other
+    block rule applies), and accepts H = 64."""
+    rng = np.random.default_rng(3)
+
+    def problem(H):
+        wg, sg = _random_mxfp4(rng, 64, 64)
+        wd, sd = _random_mxfp4(rng, 64, 64)
+        gate = np.ascontiguousarray(wg[:, : H // 2])[None]
+        gsc = np.ascontiguousarray(sg[:, : -(-H // 32)])[None]
+        return oracle.Problem(1, H, 1, 1, 64, x_dtype=oracle.F32, xq_dtype=oracle.F32, w_dtype=oracle.E2M1,
+                              h_dtype=oracle.F32, y_dtype=oracle.F32, out_dtype=oracle.F32,
+                              w_gate=gate, w_up=gate.copy(), w_down=np.ascontiguousarray(wd[:H])[None],
+                              s_gate=gsc, s_up=gsc.copy(), s_down=np.ascontiguousarray(sd[:H])[None])
+
+    x = rng.standard_normal((1, 48)).astype(np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.expert_rows(problem(48), np.zeros(1, np.int32), x)
+    x = rng.standard_normal((1, 64)).astype(np.float32)
+    h, _, y = oracle.expert_rows(problem(64), np.zeros(1, np.int32), x)
+    assert np.isfinite(y).all()
