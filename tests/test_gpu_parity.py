@@ -327,3 +327,35 @@ def test_ffn_repeated_on_one_dispatch(over, cuda_device):
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
     assert torch.equal(hs[0], hs[1]) and torch.equal(hs[1], hs[2])
     assert ys[0].abs().sum().item() > 0
+
+
+def test_dispatch_e4m3_encoder_dense_sweep(cuda_device):
+    """The dispatch kernel's e4m3 encoding against the oracle's encoder over a
+    dense sample of fp32 values in [-448, 448]: every 137th bit pattern of
+    each sign, from the subnormal range to 448 (ties, subnormals and the top
+    binade included). Each 128-value block carries +-448, so its scale is
+    exactly 1 and the stored byte is the encoding of the value itself."""
+    stride = 137
+    pos_bits = np.arange(0, 0x43E00001, stride, dtype=np.uint32)
+    vals = np.concatenate([pos_bits.view(np.float32), -pos_bits.view(np.float32)])
+    per_row = 127
+    T = -(-len(vals) // per_row)
+    x = np.zeros((T, 128), np.float32)
+    x[:, 0] = np.where(np.arange(T) % 2 == 0, 448.0, -448.0)
+    flat = np.zeros(T * per_row, np.float32)
+    flat[: len(vals)] = vals
+    x[:, 1:] = flat.reshape(T, per_row)
+    s = W.spec("sweep", T=T, H=128, E=1, k=1, act=W.F32, xq=W.E4M3, out=W.F32)
+    b = moe.alloc_buffers(s)
+    xd = torch.from_numpy(x).cuda()
+    logits = torch.zeros((T, 1), dtype=torch.float32, device="cuda")
+    moe.moe_route(b.shape, logits, b.topk_idx, b.topk_w, b.ws)
+    moe.moe_dispatch(b.shape, xd, b.topk_idx, b.ws, b.dispatch_bufs())
+    assert G.poll(b) == 0
+    pos = b.pos.cpu().numpy().astype(np.int64)
+    assert (pos >= 0).all()
+    got = b.xq[torch.from_numpy(pos).cuda()].cpu().numpy()
+    assert np.array_equal(b.xs[torch.from_numpy(pos).cuda()].cpu().numpy(), np.ones((T, 1), np.float32))
+    ref = oracle.e4m3_encode(x.astype(np.float64).ravel()).reshape(T, 128)
+    same = (got == ref) | (((got & 0x7F) == 0) & ((ref & 0x7F) == 0))   # +-0
+    assert same.all(), np.argwhere(~same)[:5]
