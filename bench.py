@@ -47,6 +47,14 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall-clock budget of the CPU oracle sample")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the prefill and MX FP4 objects of the default bench line")
+    p.add_argument("--record-traffic", default=None, metavar="NCU_CSV",
+                   help="write the DRAM bytes per launch found in an ncu --csv metrics log to "
+                        "profiles/traffic.json (with --tag and --kernel) and exit")
+    p.add_argument("--tag", default="grouped_ffn/decode")
+    p.add_argument("--kernel", default="ffn_tc_kernel")
+    p.add_argument("--how", default="")
     p.add_argument("--report", action="store_true",
                    help="instead of the single bench line: one JSON line per workload "
                         "(tiny, decode, prefill, skew, dispatch+combine sweep) with per-stage "
@@ -235,20 +243,55 @@ def ffn_flops(spec, rows):
     return 6.0 * spec.H * spec.I * rows
 
 
+TRAFFIC_JSON = os.path.join(PROFILES, "traffic.json")
+
+
 def recorded_traffic(kernel_tag: str):
-    """DRAM bytes per launch from the committed ncu summary table
-    (profiles/traffic.md), if it was taken on the current source of the
-    kernel (else None)."""
-    path = os.path.join(PROFILES, "traffic.md")
-    if not os.path.exists(path):
+    """DRAM bytes per launch of the FFN kernel for one workload, from the
+    record `python bench.py --record-traffic` wrote from an ncu capture, if
+    that capture was taken on the current source of the kernel (else None)."""
+    if not os.path.exists(TRAFFIC_JSON):
         return None
-    for line in open(path):
-        cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) >= 3 and cells[0] == kernel_tag:
-            if cells[1] != kernel_source_sha():
-                return None
-            return int(cells[2])
-    return None
+    rec = json.load(open(TRAFFIC_JSON)).get(kernel_tag)
+    if not rec or rec.get("source_sha") != kernel_source_sha():
+        return None
+    return int(rec["dram_bytes_per_launch"])
+
+
+def ncu_dram_bytes(csv_path: str, kernel_regex: str):
+    """Mean dram__bytes_read.sum + dram__bytes_write.sum per launch of the
+    kernels matching `kernel_regex` in an ncu `--csv` metrics log, and the
+    number of launches it covers."""
+    import csv
+    import re as _re
+    per = {}
+    with open(csv_path, newline="") as f:
+        rows = [r for r in csv.reader(f) if r]
+    head = next(i for i, r in enumerate(rows) if "Metric Name" in r)
+    cols = rows[head]
+    ki, mi, vi, ui, ii = (cols.index(c) for c in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit", "ID"))
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    for r in rows[head + 1:]:
+        if len(r) <= vi or not _re.search(kernel_regex, r[ki]):
+            continue
+        if r[mi] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            v = float(r[vi].replace(",", "")) * scale.get(r[ui], 1)
+            per[r[ii]] = per.get(r[ii], 0.0) + v
+    if not per:
+        raise ValueError(f"no DRAM byte metrics for {kernel_regex!r} in {csv_path}")
+    return sum(per.values()) / len(per), len(per)
+
+
+def record_traffic(args):
+    """Write one profiles/traffic.json entry from an ncu capture."""
+    mean, n = ncu_dram_bytes(args.record_traffic, args.kernel)
+    rec = json.load(open(TRAFFIC_JSON)) if os.path.exists(TRAFFIC_JSON) else {}
+    rec[args.tag] = {"source_sha": kernel_source_sha(), "dram_bytes_per_launch": int(round(mean)),
+                     "launches": n, "kernel": args.kernel, "how": args.how}
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(rec, f, indent=1, sort_keys=True)
+        f.write("\n")
+    print(json.dumps({args.tag: rec[args.tag]}))
 
 
 def kernel_source_sha() -> str:
@@ -270,33 +313,66 @@ def load_peaks():
 
 # ------------------------------------------------------------ reference --
 
+def workload_config(spec, world: int) -> dict:
+    """The `config` object of both arms' lines (one definition, so that the
+    two describe the same workload)."""
+    from combine_softmax_top_b200 import workloads as W
+    wgb = 0.0 if spec.identity else W.bytes_per_expert(spec) * spec.ne / 1e9
+    return {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
+                        f"top-{spec.k}{' + 1 shared expert' if spec.shared else ''} I={spec.I} "
+                        f"{WEIGHT_DESC.get(spec.weight, spec.weight)}",
+            "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I, "shared_experts": spec.shared,
+            "compact_windows": spec.compact,
+            "act_dtype": spec.act, "xq_dtype": spec.xq, "weight_dtype": spec.weight, "h_dtype": spec.h,
+            "y_dtype": spec.y, "out_dtype": spec.out,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed (256 MB write) before every timed step" +
+                  (f"; weights {wgb:.1f} GB > 126 MB L2" if wgb > 0.126 else "")}
+
+
 def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores, on
+    the same inputs as the GPU arm (drawn with the same generator, on the GPU
+    when there is one, then copied to the host once). One step is a bounded
+    sample of the workload: the oracle runs the layer on the first tokens
+    until the step's time budget is spent; ms_per_step is the measured wall
+    time of those steps."""
     rank, _, world = dist_env()
     if rank != 0:
         return
     from combine_softmax_top_b200 import workloads as W
     import torch
     spec = W.spec(args.config, **overrides(args))
-    inp = W.make_inputs(spec, seed=args.seed, device="cpu")
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    inp = W.make_inputs(spec, seed=args.seed, device=dev)
+    inp = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+    if dev.type == "cuda":
+        torch.cuda.empty_cache()
     per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(spec, inp, per_step / 4)
     tok = el = 0.0
     cores = 1
+    walls = []
     for _ in range(args.steps):
+        w0 = time.perf_counter()
         n, e, cores = oracle_sample(spec, inp, per_step)
+        walls.append(time.perf_counter() - w0)
         tok += n
         el += e
     value = tok / el
+    per = tok / max(1, args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * spec.T / value, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
-        "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
-                               f"top-{spec.k} I={spec.I}", "T": spec.T},
+        "ms_per_step": 1000.0 * float(statistics.mean(walls)), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64",
+        "data": f"synthetic (seeded; the GPU arm's inputs, drawn on {dev.type} and copied to the host)",
+        "config": workload_config(spec, world),
+        "step": f"a bounded sample: the layer on the first {per:.0f} of {spec.T} tokens "
+                f"(up to {per_step:.1f}s of oracle time per step)",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"first tokens of each step until {per_step:.1f}s of CPU wall time"},
+                         "sample": f"first {per:.0f} of {spec.T} tokens per step, {args.steps} steps"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -381,16 +457,18 @@ def time_e2e_pipelined(spec, inp, b, w, bufs, stream, flush, steps, dev):
     """Steps of H2D (x, logits) -> moe_layer -> D2H (out), copies overlapped
     with the neighbouring steps' layers on two copy streams (one per
     direction, so the two directions of the host link overlap too); returns
-    ms per step from the first copy to the last."""
+    ms per step from the first copy to the last. The layer is the public
+    moe_layer call with its intermediates in its own workspace."""
     import torch
     from combine_softmax_top_b200 import moe
     from combine_softmax_top_b200 import workloads as W
+    lw = moe.alloc_layer(spec, device=dev)
     hx = inp["x"].cpu().pin_memory()
     hl = inp["logits"].cpu().pin_memory()
     ho = [torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory() for _ in range(2)]
     dx = [torch.empty_like(inp["x"]) for _ in range(2)]
     dl = [torch.empty_like(inp["logits"]) for _ in range(2)]
-    dout = [b.out, torch.empty_like(b.out)]
+    dout = [lw.out, torch.empty_like(lw.out)]
     cs = torch.cuda.Stream(device=dev)        # host -> device
     co = torch.cuda.Stream(device=dev)        # device -> host
     weight_bytes = 0 if spec.identity else W.bytes_per_expert(spec) * spec.ne
@@ -419,8 +497,7 @@ def time_e2e_pipelined(spec, inp, b, w, bufs, stream, flush, steps, dev):
             stream.wait_event(ev_out[i - 2])       # out buffer i % 2 was read back
         if flush_each:
             flush.zero_()
-        moe.moe_layer(b.shape, dx[i % 2], dl[i % 2], w, b.topk_idx, b.topk_w, bufs, b.y, b.ws,
-                      dout[i % 2], stream)
+        moe.moe_layer(lw.shape, dx[i % 2], dl[i % 2], w, lw.ws, dout[i % 2], stream)
         ev_done[i].record(stream)
         with torch.cuda.stream(co):
             co.wait_event(ev_done[i])
@@ -551,6 +628,85 @@ def run_report(args):
 
 # ------------------------------------------------------------ ours --
 
+def ffn_roofline(spec, counts, ffn_ms, peaks, peak_kind, burst=True):
+    """The grouped FFN launch against both of its roofs: its algorithmic
+    bytes at the measured HBM copy rate and its FLOPs at the tensor peak of
+    its operand type (block-scaled 8-bit and 4-bit paths: twice the measured
+    bf16 GEMM rate, the nominal ratio). `bound` names the roof that is higher
+    (the slower of the two ideal times)."""
+    abytes, touched = ffn_algorithmic_bytes(spec, counts)
+    flops = ffn_flops(spec, int(counts.sum()))
+    bf16 = peaks["bf16_tflops"] if burst else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tc_peak = bf16 * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0)
+    gbs = abytes / (ffn_ms / 1000.0) / 1e9
+    tfs = flops / (ffn_ms / 1000.0) / 1e12
+    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    src = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    return {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "tensor": {"achieved": tfs, "peak": tc_peak, "unit": "TFLOP/s", "frac": tfs / tc_peak,
+                       "peak_how": ("2 x " if tc_peak != bf16 else "") +
+                                   ("burst" if burst else "sustained") + " bf16 GEMM, " + src},
+            "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                    "peak_how": "copy bandwidth, " + src},
+            "algorithmic_bytes_per_launch": abytes, "flops_per_launch": flops, "touched_experts": touched,
+            "launch_ms": ffn_ms}
+
+
+def measure_extras(args, dec_inp, dev, stream, flush, world):
+    """The other half of the metric and the 4-bit weight format, in the same
+    run as the headline decode line: the prefill layer (T = 8192, e4m3
+    weights, compact windows so the expert buffers hold 98 k rows instead of
+    2.1 M), and the decode and prefill layers with MX FP4 weights. Each is
+    timed like the headline (per-stage CUDA events on the launching stream,
+    L2 flushed before every step, clocks sampled during the timed steps).
+    The e4m3 prefill layer reuses the decode layer's weights: both draw them
+    from the same seeded streams at the same shapes."""
+    import torch
+    from combine_softmax_top_b200 import moe
+    from combine_softmax_top_b200 import workloads as W
+    peaks, peak_kind = load_peaks()
+    rank, local_rank, _ = dist_env()
+    out = {}
+    wkeys = ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
+    fp4_w = None
+    for key, name in (("prefill", "prefill"), ("decode_fp4", "decode_fp4"), ("prefill_fp4", "prefill_fp4")):
+        spec = W.spec(name, compact=1) if name.startswith("prefill") else W.spec(name)
+        inp = W.make_inputs(spec, seed=args.seed + rank, device=dev, with_weights=False)
+        if spec.weight == "e4m3":
+            inp.update({k: dec_inp[k] for k in wkeys})
+        else:
+            if fp4_w is None:
+                full = W.make_inputs(spec, seed=args.seed + rank, device=dev)
+                fp4_w = {k: v for k, v in full.items() if k in wkeys}
+                del full
+            inp.update(fp4_w)
+        b = moe.alloc_buffers(spec, device=dev)
+        clocks = ClockSampler(local_rank)
+        clocks.start()
+        st = time_layer(spec, inp, b, args.steps, args.warmup, stream, flush)
+        clk = clocks.stop()
+        mean = st.mean(0)
+        ms = max_over_ranks(float(st.sum(1).mean()), dev)
+        ffn_ms = max_over_ranks(float(mean[2]), dev)
+        counts = b.counts.cpu().numpy()
+        out[key] = {
+            "workload": workload_config(spec, world)["workload"] +
+                        (", compact windows" if spec.compact else ""),
+            "T": spec.T, "value": job_throughput(spec.T, world, ms), "unit": "tokens/s",
+            "us_per_layer": ms * 1000.0, "steps": args.steps,
+            "stage_us": {k: float(v * 1000.0) for k, v in zip(["route", "dispatch", "grouped_ffn", "combine"], mean)},
+            "roofline": ffn_roofline(spec, counts, ffn_ms, peaks, peak_kind),
+            "expert_buffer_rows": spec.rows(),
+            "l2": "flushed (256 MB write) before every timed step",
+            "clocks": clk,
+        }
+        out[key]["roofline"]["traffic"] = recorded_traffic(f"grouped_ffn/{spec.name}")
+        del inp, b
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -651,26 +807,20 @@ def run_ours(args):
     ffn_ms = float(stage[:, 2].mean())
     roofline = None
     if not spec.identity:
-        abytes, touched = ffn_algorithmic_bytes(spec, counts)
-        flops = ffn_flops(spec, int(counts.sum()))
-        bw = abytes / (ffn_ms / 1000.0) / 1e9
         # decode-size GEMMs stream weights (HBM bound); big-batch GEMMs are
-        # bound by the tensor pipe
-        t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
-        t_tc = flops / (peaks["bf16_tflops"] * 1e12 * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0))
-        if t_hbm >= t_tc:
-            roofline = {"bound": "hbm", "achieved": bw, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": bw / peaks["hbm_gbs"]}
-        else:
-            pk = peaks["bf16_tflops"] * (2.0 if spec.weight in ("e4m3", "e2m1") else 1.0)
-            ach = flops / (ffn_ms / 1000.0) / 1e12
-            roofline = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
-                        "frac": ach / pk}
-        roofline.update({"kernel": "grouped_ffn", "algorithmic_bytes_per_launch": abytes,
-                         "flops_per_launch": flops, "touched_experts": touched,
-                         "launch_ms": ffn_ms, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
-                         if peak_kind == "measured" else "fallback",
-                         "traffic": recorded_traffic(f"grouped_ffn/{spec.name}")})
+        # bound by the tensor pipe: the headline keys name the higher roof
+        both = ffn_roofline(spec, counts, ffn_ms, peaks, peak_kind)
+        top = both[both["bound"]]
+        roofline = {"bound": both["bound"], "achieved": top["achieved"], "peak": top["peak"],
+                    "unit": top["unit"], "frac": top["frac"], "kernel": "grouped_ffn",
+                    "algorithmic_bytes_per_launch": both["algorithmic_bytes_per_launch"],
+                    "flops_per_launch": both["flops_per_launch"], "touched_experts": both["touched_experts"],
+                    "launch_ms": ffn_ms, "peak_source": top["peak_how"],
+                    "traffic": recorded_traffic(f"grouped_ffn/{spec.name}")}
+
+    extras = {}
+    if args.config == "decode" and not overrides(args) and not args.no_extra:
+        extras = measure_extras(args, inp, dev, stream, flush, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -689,13 +839,7 @@ def run_ours(args):
             "us_per_layer": ms * 1000.0, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if spec.weight == "e4m3" else spec.weight,
             "data": "synthetic (seeded; random-init weights, no checkpoint)",
-            "config": {"workload": f"{spec.name} MoE layer T={spec.T} H={spec.H} E={spec.E} "
-                                   f"top-{spec.k}{' + 1 shared expert' if spec.shared else ''} I={spec.I} "
-                                   f"{WEIGHT_DESC.get(spec.weight, spec.weight)}",
-                       "T": spec.T, "H": spec.H, "E": spec.E, "topk": spec.k, "I": spec.I, "shared_experts": spec.shared,
-                       "compact_windows": spec.compact,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed (256 MB write) before every timed step; weights 11 GB > L2"},
+            "config": workload_config(spec, world),
             "stage_us": {k: float(stage[:, j].mean() * 1000.0)
                          for j, k in enumerate(["route", "dispatch", "grouped_ffn", "combine"])},
             "roofline": roofline,
@@ -705,6 +849,7 @@ def run_ours(args):
             "gpu_launches": args.steps * moe.kernels_per_layer(spec),
             "clocks": clk,
         }
+        line.update(extras)
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
@@ -712,7 +857,9 @@ def run_ours(args):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.record_traffic:
+        record_traffic(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.report:
         run_report(args)

@@ -32,12 +32,15 @@
 // launches): plan_kernel histograms the expert indices and its last CTA
 // lays the windows out back to back, each rounded up to whole 128-row tiles,
 // so the buffers need T * k + 127 * E rows instead of E * cap.
+#include <atomic>
+
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kMaxDevices = 64;   // per-device caches of launch parameters
 constexpr int kElems = 16;  // values per lane per step
 
 struct Args {
@@ -468,17 +471,24 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
     if (err != cudaSuccess) return err;
   }
   // one wave of resident CTAs, each walking several tokens (fewer CTAs also
-  // means fewer arrivals on the closing counter)
-  auto go = [&](auto kern, int& resident) {
+  // means fewer arrivals on the closing counter). The occupancy query is
+  // cached per device and kernel; concurrent callers may both run it, and
+  // they store the same value.
+  auto go = [&](auto kern, std::atomic<int>* cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return;
+    std::atomic<int>& slot = cache[dev >= 0 && dev < kMaxDevices ? dev : 0];
+    int resident = (dev >= 0 && dev < kMaxDevices) ? slot.load(std::memory_order_relaxed) : 0;
     if (resident == 0) {
       int r = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kThreads, 0) != cudaSuccess || r < 1) r = 1;
       resident = r;
+      if (dev >= 0 && dev < kMaxDevices) slot.store(r, std::memory_order_relaxed);
     }
     const int grid = a.T > 0 ? std::min(a.T, c.num_sms * resident) : 1;
     kern<<<grid, kThreads, 0, c.stream>>>(a);
   };
-  static int resident_bf16 = 0, resident_f32 = 0;
+  static std::atomic<int> resident_bf16[kMaxDevices], resident_f32[kMaxDevices];
   if (a.act == MOE_BF16) go(dispatch_kernel<MOE_BF16>, resident_bf16);
   else go(dispatch_kernel<MOE_F32>, resident_f32);
   return cudaGetLastError();

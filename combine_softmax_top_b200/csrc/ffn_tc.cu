@@ -205,6 +205,15 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.f + expf
 // UE8M0 code of a power-of-two fp32 scale: its biased exponent.
 __device__ __forceinline__ uint32_t ue8m0(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
+// A weight block scale the block-scaled MMA applies exactly: a positive,
+// finite, normal power of two (sign and mantissa bits zero, exponent neither
+// 0 nor 255). Any other value would lose its mantissa in ue8m0().
+__device__ __forceinline__ bool pow2_scale_ok(float s) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t e = (b >> 23) & 0xFFu;
+  return (b & 0x807FFFFFu) == 0u && e != 0u && e != 0xFFu;
+}
+
 template <int kW, int kBRows>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool kFp8 = kW != kWBf16;   // block-scaled MMA, e4m3 tokens
@@ -471,13 +480,27 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         atom_b = down ? atom_a + (int64_t)nkb * kSfAtomBytes
                       : (const uint8_t*)p.su + ((int64_t)j.e * n_out + j.slice) * nkb * kSfAtomBytes;
       }
+      // A scale that is not a normal power of two latches
+      // MOE_ERR_INVALID_ARG (info: 0x25, the matrix (0 gate / down, 1 up or
+      // the second down slice) and the expert); the layer's outputs are then
+      // unspecified. Every scale of every touched expert passes through here.
       auto load_scales = [&](int base) {
-        if (lane + base < nkb) sa0 = ue8m0(__ldg(pa + base + lane));
-        if (lane + base + 32 < nkb) sa1 = ue8m0(__ldg(pa + base + lane + 32));
+        bool bad = false;
+        auto take = [&](const float* src, int kb) -> uint32_t {
+          const float v = __ldg(src + kb);
+          bad |= !pow2_scale_ok(v);
+          return ue8m0(v);
+        };
+        if (lane + base < nkb) sa0 = take(pa, base + lane);
+        if (lane + base + 32 < nkb) sa1 = take(pa, base + lane + 32);
+        const bool bad_a = bad;
         if (dual) {
-          if (lane + base < nkb) sb0 = ue8m0(__ldg(pb + base + lane));
-          if (lane + base + 32 < nkb) sb1 = ue8m0(__ldg(pb + base + lane + 32));
+          if (lane + base < nkb) sb0 = take(pb, base + lane);
+          if (lane + base + 32 < nkb) sb1 = take(pb, base + lane + 32);
         }
+        const uint32_t which = __ballot_sync(0xffffffffu, bad_a) ? 0u : 1u;
+        if (__ballot_sync(0xffffffffu, bad) != 0u && lane == 0)
+          latch_error(hdr, MOE_ERR_INVALID_ARG, 0x25000000u | (which << 20) | (uint32_t)j.e);
       };
       // the four exponents of blocks kr .. kr+3 (relative to sbase), packed
       auto pack4 = [&](uint32_t r0, uint32_t r1, int kr) -> uint32_t {

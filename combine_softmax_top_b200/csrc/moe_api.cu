@@ -91,6 +91,43 @@ moe_status make_ctx(const moe_shape* s, void* ws, moe_stream_t stream, Ctx* c) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// The intermediates moe_layer keeps in its workspace, after the stage
+// workspace (Layout::total): topk_idx, topk_w, the dispatch buffers and y,
+// each 256-byte aligned. rows = E * cap (or the compact bound) of the
+// effective shape.
+struct LayerState {
+  size_t off_idx, off_w, off_xq, off_xs, off_counts, off_offsets, off_row_src, off_pos, off_hq, off_hs, off_y;
+  size_t total;
+};
+
+size_t dtype_bytes(int32_t d) { return d == MOE_F32 ? 4 : (d == MOE_BF16 ? 2 : 1); }
+
+LayerState layer_state(const moe_shape& s, const Layout& L) {
+  LayerState st{};
+  const size_t rows = (size_t)L.tiles * kTileRows;
+  const size_t pairs = (size_t)s.T * (size_t)s.topk;
+  size_t off = L.total;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  st.off_idx = take(pairs * 4);
+  st.off_w = take(pairs * 4);
+  st.off_xq = take(rows * (size_t)s.H * dtype_bytes(s.xq_dtype));
+  st.off_xs = take(s.xq_dtype == MOE_E4M3 ? rows * (size_t)(s.H / kQBlock) * 4 : 0);
+  st.off_counts = take((size_t)s.E * 4);
+  st.off_offsets = take((size_t)s.E * 4);
+  st.off_row_src = take(rows * 4);
+  st.off_pos = take(pairs * 4);
+  const bool ffn = !s.identity_experts;
+  st.off_hq = take(ffn ? rows * (size_t)s.I * dtype_bytes(s.h_dtype) : 0);
+  st.off_hs = take(ffn && s.h_dtype == MOE_E4M3 ? rows * (size_t)(s.I / kQBlock) * 4 : 0);
+  st.off_y = take(ffn ? rows * (size_t)s.H * dtype_bytes(s.y_dtype) : 0);
+  st.total = off;
+  return st;
+}
+
 }  // namespace
 
 moe_status check_bufs(const moe_shape* s, const moe_dispatch_bufs* b, bool need_h) {
@@ -223,9 +260,39 @@ moe_status moe_combine(const moe_shape* shape, const moe_dispatch_bufs* bufs, co
   return st != MOE_OK ? st : do_combine(c, bufs, y, topk_w, out);
 }
 
+moe_status moe_layer_workspace_bytes(const moe_shape* shape, size_t* bytes) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const moe_shape e = effective_shape(*shape);
+  *bytes = layer_state(e, make_layout(e)).total;
+  return MOE_OK;
+}
+
 moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,
-                     int32_t* topk_idx, float* topk_w, const moe_dispatch_bufs* bufs, void* y,
                      void* ws, void* out, moe_stream_t stream) {
+  Ctx c;
+  moe_status st = make_ctx(shape, ws, stream, &c);
+  if (st != MOE_OK) return st;
+  const LayerState ls = layer_state(c.s, c.L);
+  char* b = (char*)ws;
+  moe_dispatch_bufs bufs;
+  bufs.xq = b + ls.off_xq;
+  bufs.xs = c.s.xq_dtype == MOE_E4M3 ? (float*)(b + ls.off_xs) : nullptr;
+  bufs.counts = (int32_t*)(b + ls.off_counts);
+  bufs.offsets = (int32_t*)(b + ls.off_offsets);
+  bufs.row_src = (int32_t*)(b + ls.off_row_src);
+  bufs.pos = (int32_t*)(b + ls.off_pos);
+  bufs.hq = c.s.identity_experts ? nullptr : (void*)(b + ls.off_hq);
+  bufs.hs = (!c.s.identity_experts && c.s.h_dtype == MOE_E4M3) ? (float*)(b + ls.off_hs) : nullptr;
+  void* y = c.s.identity_experts ? nullptr : (void*)(b + ls.off_y);
+  return moe_layer_bufs(shape, x, logits, w, (int32_t*)(b + ls.off_idx), (float*)(b + ls.off_w), &bufs, y, ws,
+                        out, stream);
+}
+
+moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,
+                          int32_t* topk_idx, float* topk_w, const moe_dispatch_bufs* bufs, void* y,
+                          void* ws, void* out, moe_stream_t stream) {
   Ctx c;
   moe_status st = make_ctx(shape, ws, stream, &c);
   if (st != MOE_OK) return st;

@@ -25,8 +25,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CAPACITY", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_NONFINITE"}
 
 EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
-           "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_poll_status", "moe_status_string",
-           "moe_dispatch_noalloc", "moe_pack_mx_scales")
+           "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_layer_bufs", "moe_layer_workspace_bytes",
+           "moe_poll_status", "moe_status_string", "moe_dispatch_noalloc", "moe_pack_mx_scales")
 
 
 class MoeError(RuntimeError):
@@ -77,8 +77,10 @@ def lib() -> ctypes.CDLL:
             "moe_grouped_ffn": [S, ctypes.POINTER(moe_dispatch_bufs), ctypes.POINTER(moe_weights),
                                 P, P, P],
             "moe_combine": [S, ctypes.POINTER(moe_dispatch_bufs), P, P, P, P, P],
-            "moe_layer": [S, P, P, ctypes.POINTER(moe_weights), P, P,
-                          ctypes.POINTER(moe_dispatch_bufs), P, P, P, P],
+            "moe_layer": [S, P, P, ctypes.POINTER(moe_weights), P, P, P],
+            "moe_layer_bufs": [S, P, P, ctypes.POINTER(moe_weights), P, P,
+                               ctypes.POINTER(moe_dispatch_bufs), P, P, P, P],
+            "moe_layer_workspace_bytes": [S, ctypes.POINTER(ctypes.c_size_t)],
             "moe_poll_status": [P, P],
             "moe_dispatch_noalloc": [S, P, P, ctypes.POINTER(moe_dispatch_bufs), P],
             "moe_status_string": [ctypes.c_int],
@@ -158,12 +160,26 @@ def moe_combine(shape, bufs: moe_dispatch_bufs, y, topk_w, ws, out, stream=None)
                                             _ptr(topk_w), _ptr(ws), _ptr(out), _stream(stream)))
 
 
-def moe_layer(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe_dispatch_bufs, y, ws,
-              out, stream=None) -> None:
+def moe_layer_workspace_bytes(shape: moe_shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_layer_workspace_bytes",
+           lib().moe_layer_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def moe_layer(shape, x, logits, w: moe_weights, ws, out, stream=None) -> None:
+    """The whole layer with every intermediate inside `ws` (of at least
+    moe_layer_workspace_bytes bytes)."""
     _check("moe_layer", lib().moe_layer(ctypes.byref(shape), _ptr(x), _ptr(logits),
-                                        ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
-                                        ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
-                                        _stream(stream)))
+                                        ctypes.byref(w), _ptr(ws), _ptr(out), _stream(stream)))
+
+
+def moe_layer_bufs(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe_dispatch_bufs, y, ws,
+                   out, stream=None) -> None:
+    _check("moe_layer_bufs", lib().moe_layer_bufs(ctypes.byref(shape), _ptr(x), _ptr(logits),
+                                                  ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
+                                                  ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
+                                                  _stream(stream)))
 
 
 def moe_pack_mx_scales(src: torch.Tensor, stream=None) -> torch.Tensor:
@@ -265,10 +281,33 @@ def weights_struct(inp: dict) -> moe_weights:
 
 
 def run_layer(b: Buffers, inp: dict, stream=None) -> None:
-    """Enqueue one whole layer (moe_layer) on the current stream."""
+    """Enqueue one whole layer into `b`'s buffers (moe_layer_bufs) on the
+    current stream."""
     w = weights_struct(inp) if not b.spec.identity else moe_weights()
-    moe_layer(b.shape, inp["x"], inp["logits"], w, b.topk_idx, b.topk_w, b.dispatch_bufs(), b.y,
-              b.ws, b.out, stream)
+    moe_layer_bufs(b.shape, inp["x"], inp["logits"], w, b.topk_idx, b.topk_w, b.dispatch_bufs(), b.y,
+                   b.ws, b.out, stream)
+
+
+@dataclass
+class LayerWorkspace:
+    """A workspace holding every intermediate of moe_layer, and the output."""
+    shape: moe_shape
+    spec: Spec
+    ws: torch.Tensor
+    out: torch.Tensor
+
+
+def alloc_layer(s: Spec, device="cuda", stream=None) -> LayerWorkspace:
+    sh = make_shape(s)
+    ws = torch.empty(moe_layer_workspace_bytes(sh), dtype=torch.uint8, device=device)
+    moe_workspace_init(sh, ws, stream)
+    return LayerWorkspace(sh, s, ws, torch.empty((s.T, s.H), dtype=_TORCH[s.out], device=device))
+
+
+def run_layer_ws(lw: LayerWorkspace, inp: dict, stream=None) -> None:
+    """Enqueue one whole layer (moe_layer, intermediates in the workspace)."""
+    w = weights_struct(inp) if not lw.spec.identity else moe_weights()
+    moe_layer(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, stream)
 
 
 # kernels the library launches per stage (mirrors the launch plan in csrc/)

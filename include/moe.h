@@ -172,7 +172,10 @@ typedef struct moe_dispatch_bufs {
  *   w_gate, w_up [E, I, H]; w_down [E, H, I], in weight_dtype.
  *   E4M3 weights carry one fp32 scale per 128 x 128 block:
  *   s_gate, s_up [E, I/128, H/128]; s_down [E, H/128, I/128]. Scales must be
- *   powers of two (the tensor cores apply them as 8-bit exponents).
+ *   positive, finite, normal powers of two (the tensor cores apply them as
+ *   8-bit exponents): moe_grouped_ffn checks every scale it uses and latches
+ *   MOE_ERR_INVALID_ARG for any other value (the outputs are then
+ *   unspecified), rather than dropping its mantissa.
  *   E2M1 weights hold two 4-bit codes per byte, element 2i of a row in the
  *   low nibble of its byte i (w_gate, w_up [E, I, H/2] bytes; w_down
  *   [E, H, I/2]; each matrix 32-byte aligned), and one UE8M0 scale byte
@@ -270,11 +273,40 @@ MOE_API moe_status moe_combine(const moe_shape* shape, const moe_dispatch_bufs* 
                        const float* topk_w, void* ws, void* out, moe_stream_t stream);
 
 /*
- * The whole layer: moe_route, moe_dispatch, moe_grouped_ffn, moe_combine
- * enqueued in that order on `stream`. Intermediates go to the caller's
- * buffers (topk_idx/topk_w [T, topk], bufs, y) so that they can be inspected.
+ * Size in bytes of a workspace that moe_layer can use (host only): the stage
+ * workspace of moe_workspace_bytes followed by room for the layer's
+ * intermediates (topk_idx, topk_w, the expert-major buffers of
+ * moe_dispatch_bufs and y, at the sizes given there; with MOE_FLAG_COMPACT
+ * the buffers are the compact bound, about T * topk rows, else E * cap rows).
+ */
+MOE_API moe_status moe_layer_workspace_bytes(const moe_shape* shape, size_t* bytes);
+
+/*
+ * The whole layer (route, one-pass dispatch, grouped expert FFN, combine),
+ * enqueued in that order on `stream`; the pages' problem statement in one
+ * call (GC-MoE explainer, "Why Expert Parallelism Is Inefficient in MoE
+ * Decoding": an MoE layer is gating, token dispatch, the experts' GEMMs and a
+ * combine back to token order).
+ *   x       [T, H] act_dtype, device
+ *   logits  [T, E] fp32, device
+ *   w       expert weights (as for moe_grouped_ffn; ignored with identity
+ *           experts)
+ *   ws      device workspace of at least moe_layer_workspace_bytes bytes,
+ *           256-byte aligned and prepared by moe_workspace_init; every
+ *           intermediate lives in it (the size cannot be checked here: a
+ *           smaller buffer is the caller's error)
+ *   out     [T, H] out_dtype, device
+ * Errors as for the four stages; device errors latch into ws.
  */
 MOE_API moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits,
+                     const moe_weights* w, void* ws, void* out, moe_stream_t stream);
+
+/*
+ * moe_layer with the intermediates in the caller's own buffers
+ * (topk_idx/topk_w [T, topk], bufs, y, as for the stage calls), so that they
+ * can be inspected or kept; ws needs only moe_workspace_bytes bytes.
+ */
+MOE_API moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const float* logits,
                      const moe_weights* w, int32_t* topk_idx, float* topk_w,
                      const moe_dispatch_bufs* bufs, void* y, void* ws, void* out,
                      moe_stream_t stream);
@@ -287,15 +319,24 @@ MOE_API moe_status moe_layer(const moe_shape* shape, const void* x, const float*
  * an allocation brings). The pages have no counterpart of this call.
  *
  * Arguments and outputs are those of moe_dispatch (bufs: xq, xs, counts,
- * offsets, row_src, pos). The dispatch kernel's own state lives instead in a
- * fixed 4 MiB array of device memory inside the library, which every GPU that
- * loads the library holds until the process exits; a shape whose workspace
- * (moe_workspace_bytes) exceeds 4 MiB is rejected with MOE_ERR_INVALID_ARG.
- * The first call on each device looks up that array's device address (with
- * the device current), so make it before any stream capture. Every call
- * clears what the kernel needs zeroed, then dispatches; calls that overlap on
- * the GPU share the array and race. Device-detected errors are not reported
- * through a workspace: a pair that could not be placed has pos = -1.
+ * offsets, row_src, pos). The dispatch kernel's own state (counters, tile
+ * sentinels and the tile ring) lives instead in a fixed 4 MiB array of device
+ * memory inside the library, which every GPU that loads the library holds
+ * until the process exits; a shape whose counters, sentinels and ring need
+ * more than 4 MiB is rejected with MOE_ERR_INVALID_ARG (the scale atoms that
+ * moe_dispatch also writes into its workspace are not made here, so they do
+ * not count). The first call on each device looks up that array's device
+ * address (with the device current), so make it before any stream capture.
+ * Every call clears what the kernel needs zeroed, then dispatches; calls that
+ * overlap on the GPU share the array and race. Device-detected errors are not
+ * reported through a workspace: a pair that could not be placed has pos = -1.
+ *
+ * Its outputs may be read by the host or passed to moe_combine with identity
+ * experts (identity_experts = 1, which reads xq/xs through pos). They must
+ * not be passed to moe_grouped_ffn or moe_layer: those read the tile
+ * sentinels, ring and scale atoms from their workspace, which this call does
+ * not write, and a workspace that an earlier moe_dispatch used would hand them
+ * stale ones.
  */
 MOE_API moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                                         const moe_dispatch_bufs* bufs, moe_stream_t stream);

@@ -152,3 +152,32 @@ def test_pack_mx_scales_rejects_bad_sizes(n, rows, cols):
 
 def test_pack_mx_scales_empty_enqueues_nothing():
     assert moe.lib().moe_pack_mx_scales(0, 128, 128, None, None, None) == 0
+
+
+def test_layer_workspace_holds_the_intermediates():
+    """moe_layer keeps topk_idx/topk_w, the expert-major buffers and y after
+    the stage workspace: its size is at least the stage workspace plus those
+    arrays at the sizes moe.h gives for them."""
+    for s in (W.spec("decode"), W.spec("prefill", compact=1), W.spec("tiny"), W.spec("sweep"),
+              W.spec("decode", shared=1)):
+        sh = moe.make_shape(s)
+        stage = moe.moe_workspace_bytes(sh)
+        layer = moe.moe_layer_workspace_bytes(sh)
+        el = {"f32": 4, "bf16": 2, "e4m3": 1}
+        rows = s.rows()
+        need = 2 * s.T * s.ks * 4 + rows * s.H * el[s.xq] + rows * 4 + s.T * s.ks * 4
+        if not s.identity:
+            need += rows * s.I * el[s.h] + rows * s.H * el[s.y]
+        assert layer >= stage + need, s.name
+        assert layer % 256 == 0
+
+
+def test_layer_checks_arguments_before_any_launch():
+    sh = moe.make_shape(W.spec("decode"))
+    L = moe.lib()
+    assert L.moe_layer(ctypes.byref(sh), None, None, None, None, None, None) == 1
+    bad = moe.make_shape(W.spec("decode"))
+    bad.topk = 0
+    n = ctypes.c_size_t(0)
+    assert L.moe_layer_workspace_bytes(ctypes.byref(bad), ctypes.byref(n)) == 1
+    assert L.moe_layer_workspace_bytes(ctypes.byref(sh), None) == 1

@@ -359,3 +359,51 @@ def test_dispatch_e4m3_encoder_dense_sweep(cuda_device):
     ref = oracle.e4m3_encode(x.astype(np.float64).ravel()).reshape(T, 128)
     same = (got == ref) | (((got & 0x7F) == 0) & ((ref & 0x7F) == 0))   # +-0
     assert same.all(), np.argwhere(~same)[:5]
+
+
+# ------------------------------------------- the workspace-only layer call --
+
+@pytest.mark.parametrize("name,over", [
+    ("decode", dict(T=32, H=512, E=16, k=4, I=256)),
+    ("decode", dict(T=300, H=512, E=4, k=2, I=384, compact=1)),
+    ("tiny", {}),
+])
+def test_layer_with_intermediates_in_workspace(name, over, cuda_device):
+    """moe_layer (every intermediate carved from its workspace) gives the same
+    bytes as moe_layer_bufs (the caller's buffers) on the same inputs: the
+    layer output is bitwise stable run to run."""
+    s = W.spec(name, **over)
+    inp = W.make_inputs(s, seed=7, device="cuda")
+    b = G.run_stages(s, inp, layer=True)
+    assert G.poll(b) == 0
+    lw = moe.alloc_layer(s)
+    for _ in range(2):                          # two calls on one workspace
+        moe.run_layer_ws(lw, inp)
+        torch.cuda.synchronize()
+        assert moe.moe_poll_status(lw.ws) == 0
+        assert torch.equal(lw.out, b.out)
+
+
+# ------------------------------------------------ weight scale precondition --
+
+@pytest.mark.parametrize("bad", [0.75, -1.0, 0.0, float("inf"), float("nan"), 2.0 ** -130])
+@pytest.mark.parametrize("over", [dict(T=32, H=512, E=16, k=4, I=256), dict(T=16, H=512, E=32, k=4, I=256)])
+def test_weight_scales_that_are_not_powers_of_two_are_refused(bad, over, cuda_device):
+    """The block-scaled MMA applies a weight scale as an 8-bit exponent; a
+    scale it cannot apply exactly (a mantissa, a sign, zero, inf, NaN, a
+    subnormal) is refused on the device with MOE_ERR_INVALID_ARG instead of
+    being truncated, whichever matrix holds it. A power of two passes."""
+    s = W.spec("decode", **over)
+    inp = W.make_inputs(s, seed=8, device="cuda")
+    for name in ("s_gate", "s_up", "s_down"):
+        case = dict(inp)
+        sc = inp[name].clone()
+        # a mantissa or a sign on a valid scale; zero, inf, NaN, a subnormal as is
+        sc[:, 0, 1] = sc[:, 0, 1] * bad if bad in (0.75, -1.0) else torch.full_like(sc[:, 0, 1], bad)
+        case[name] = sc
+        b = G.run_stages(s, case)
+        assert G.poll(b) == 1, (name, bad)      # MOE_ERR_INVALID_ARG
+    ok = dict(inp)
+    ok["s_up"] = inp["s_up"] * 2.0
+    b = G.run_stages(s, ok)
+    assert G.poll(b) == 0

@@ -11,6 +11,8 @@ checked, since every call reuses the library's one fixed scratch array.
 This file is named to be collected last: if it fails, a run that stops at the
 first failure has already run every other test.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -38,6 +40,7 @@ def _assert_same_dispatch(got, ref, s):
     assert np.array_equal(got["offsets"], ref["offsets"])
     cap = s.cap
     gp, rp = got["pos"], ref["pos"]
+    assert len(gp) == s.T * s.ks
     assert np.array_equal(gp >= 0, rp >= 0)
     placed = np.nonzero(rp >= 0)[0]
     # same expert window for every pair, and row_src pointing back at it
@@ -53,6 +56,9 @@ def _assert_same_dispatch(got, ref, s):
 @pytest.mark.parametrize("name,over", [
     ("decode", {}),                                     # e4m3 rows, 128 tokens
     ("skew", dict(T=256, H=1024, E=32)),                # bf16 rows, skewed counts
+    ("tiny", {}),                                       # fp32 rows
+    # a shared expert: every token's extra slot goes to expert E of E + 1
+    ("decode", dict(T=32, H=512, E=16, k=4, I=256, shared=1)),
 ])
 def test_noalloc_dispatch_matches_workspace_dispatch(name, over, cuda_device):
     s = W.spec(name, **over)
@@ -78,3 +84,71 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_dispatch_noalloc(sh, b.out, b.topk_idx, b.dispatch_bufs())
     assert ei.value.code == 1                           # MOE_ERR_INVALID_ARG
+
+
+def _bound_T(E: int) -> int:
+    """The smallest multiple of 128 tokens whose counters, sentinels and ring
+    (the whole workspace of a bf16 layer with identity experts, which has no
+    scale atoms) need more than the 4 MiB the no-workspace dispatch has."""
+    T = 128
+    while moe.moe_workspace_bytes(moe.make_shape(W.spec("skew", T=T, E=E, H=16, identity=1))) <= 4 << 20:
+        T += 128
+    return T
+
+
+def test_noalloc_rejects_a_shape_just_over_its_scratch():
+    """Refused on the host before any CUDA call (so this runs without a GPU;
+    the pointers are never looked at)."""
+    T = _bound_T(1024)
+    sh = moe.make_shape(W.spec("skew", T=T, E=1024, H=16, identity=1))
+    fake = ctypes.c_void_p(1 << 20)
+    b = moe.moe_dispatch_bufs()
+    for f, _ in b._fields_:
+        setattr(b, f, 1 << 20)
+    assert moe.lib().moe_dispatch_noalloc(ctypes.byref(sh), fake, fake, ctypes.byref(b), None) == 1
+
+
+def test_noalloc_accepts_a_shape_just_under_its_scratch(cuda_device):
+    T = _bound_T(1024) - 128
+    s = W.spec("skew", T=T, E=1024, H=16, identity=1)   # 16 values per token keep the windows small
+    inp = W.make_inputs(s, seed=3, device="cuda", with_weights=False)
+    ref = moe.alloc_buffers(s)
+    moe.moe_route(ref.shape, inp["logits"], ref.topk_idx, ref.topk_w, ref.ws)
+    moe.moe_dispatch(ref.shape, inp["x"], ref.topk_idx, ref.ws, ref.dispatch_bufs())
+    assert moe.moe_poll_status(ref.ws) == 0
+    got = moe.alloc_buffers(s)
+    moe.moe_dispatch_noalloc(got.shape, inp["x"], ref.topk_idx, got.dispatch_bufs())
+    _assert_same_dispatch(_dispatch_outputs(got), _dispatch_outputs(ref), s)
+
+
+def test_noalloc_accepts_prefill_token_and_expert_counts(cuda_device):
+    """T = 8192 over 256 experts (the prefill layer's counts, with a small
+    hidden size): 0.5 MB of counters, sentinels and ring."""
+    s = W.spec("prefill", H=512, I=256)
+    inp = W.make_inputs(s, seed=4, device="cuda", with_weights=False)
+    ref = moe.alloc_buffers(s)
+    moe.moe_route(ref.shape, inp["logits"], ref.topk_idx, ref.topk_w, ref.ws)
+    moe.moe_dispatch(ref.shape, inp["x"], ref.topk_idx, ref.ws, ref.dispatch_bufs())
+    assert moe.moe_poll_status(ref.ws) == 0
+    got = moe.alloc_buffers(s)
+    moe.moe_dispatch_noalloc(got.shape, inp["x"], ref.topk_idx, got.dispatch_bufs())
+    _assert_same_dispatch(_dispatch_outputs(got), _dispatch_outputs(ref), s)
+
+
+def test_noalloc_outputs_feed_identity_combine(cuda_device):
+    """What the no-workspace dispatch writes is enough for moe_combine with
+    identity experts: the output equals the oracle's identity layer (the
+    dequantised token, weights summing to one) within one bf16 rounding."""
+    import oracle
+    from tests import gpu_harness as G
+    from tests.helpers import as_f64, raw
+    s = W.spec("sweep", T=512)
+    inp = W.make_inputs(s, seed=6, device="cuda")
+    b = moe.alloc_buffers(s)
+    moe.moe_route(b.shape, inp["logits"], b.topk_idx, b.topk_w, b.ws)
+    moe.moe_dispatch_noalloc(b.shape, inp["x"], b.topk_idx, b.dispatch_bufs())
+    moe.moe_combine(b.shape, b.dispatch_bufs(), None, b.topk_w, b.ws, b.out)
+    assert moe.moe_poll_status(b.ws) == 0
+    r = oracle.moe_layer(G.oracle_problem(s, inp), raw(inp["x"]), raw(inp["logits"]))
+    out, ref = as_f64(raw(b.out), "bf16"), as_f64(r["out"], "bf16")
+    assert np.all(np.abs(out - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-30)
