@@ -55,6 +55,9 @@ def parse():
     p.add_argument("--tag", default="grouped_ffn/decode")
     p.add_argument("--kernel", default="ffn_tc_kernel")
     p.add_argument("--how", default="")
+    p.add_argument("--overlap-sweep", action="store_true",
+                   help="print one JSON line per workload (decode, prefill on compact windows) timing "
+                        "the layer with dispatch beside the grouped FFN over a sweep of partition sizes")
     p.add_argument("--report", action="store_true",
                    help="instead of the single bench line: one JSON line per workload "
                         "(tiny, decode, prefill, skew, dispatch+combine sweep) with per-stage "
@@ -560,6 +563,105 @@ def time_whole_layer(spec, inp, b, steps, warmup, flush):
     return stream_ms, graph_ms
 
 
+def time_overlap(spec, inp, dev, flush, steps, warmup, splits=(8, 20, 32), green=(20,)):
+    """The whole layer with dispatch beside the grouped FFN (moe_layer_overlap)
+    against the same layer run stage after stage (moe_layer), both with their
+    intermediates in a layer workspace, L2 flushed before every timed step,
+    median device time on the launching stream (the join makes that stream
+    wait for the dispatch stream, so the interval covers both). Each split
+    gives dispatch P SMs' worth of CTAs and the FFN's persistent grid the
+    other SMs; it is timed stream-launched and as the replay of a CUDA graph
+    of one call (route and the counting pass, then dispatch and the FFN as
+    two concurrent branches, then combine). `green` splits put the dispatch
+    stream in a green context of P SMs instead."""
+    import numpy as np
+    import torch
+    from combine_softmax_top_b200 import moe
+
+    lw = moe.alloc_layer(spec, device=dev)
+    w = moe.weights_struct(inp)
+
+    def timed(fn):
+        for _ in range(max(3, warmup)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        rc = moe.moe_poll_status(lw.ws)
+        if rc != 0:
+            raise RuntimeError(f"layer reported {moe.moe_status_string(rc)}")
+        return float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+
+    def graphed(fn):
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        ms = timed(g.replay)
+        del g
+        return ms
+
+    def serial():
+        moe.moe_layer(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out)
+
+    res = {"serial_us": timed(serial) * 1e3, "serial_graph_us": graphed(serial) * 1e3, "splits": {}}
+    ref = lw.out.clone()
+    for P, is_green in [(P, False) for P in splits] + [(P, True) for P in green]:
+        key = f"{P}" + ("_green" if is_green else "")
+        try:
+            ov = moe.Overlap(P, green=is_green, device=dev)
+        except Exception as exc:   # torch without green contexts, or the driver refuses one
+            res["splits"][key] = {"unavailable": str(exc)[:200]}
+            continue
+
+        def over(ov=ov):
+            moe.moe_layer_overlap(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, ov.ov)
+
+        try:
+            r = {"us": timed(over) * 1e3, "graph_us": graphed(over) * 1e3}
+        except Exception as exc:
+            r = {"unavailable": str(exc)[:200]}
+        else:
+            r["same_bits"] = bool(torch.equal(lw.out, ref))
+        res["splits"][key] = r
+    best = min((v["us"], k) for k, v in res["splits"].items() if "us" in v)
+    res["best"] = {"split": best[1], "us": best[0], "gain_vs_serial": res["serial_us"] / best[0]}
+    res["how"] = ("moe_layer vs moe_layer_overlap on a layer workspace; median of the timed steps, "
+                  "L2 flushed before each; split = SMs sized for dispatch, the FFN grid the rest")
+    del lw
+    return res
+
+
+def run_overlap_sweep(args):
+    import torch
+    from combine_softmax_top_b200 import workloads as W
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for spec in (W.spec("decode"), W.spec("prefill", compact=1), W.spec("decode_fp4")):
+        inp = W.make_inputs(spec, seed=args.seed, device=dev)
+        clocks = ClockSampler(0)
+        clocks.start()
+        r = time_overlap(spec, inp, dev, flush, args.steps, args.warmup,
+                         splits=(2, 4, 8, 12, 16, 20, 24, 32, 48), green=(8, 20))
+        r["clocks"] = clocks.stop()
+        r["workload"] = workload_config(spec, 1)["workload"] + (", compact windows" if spec.compact else "")
+        print(json.dumps(r), flush=True)
+        del inp
+        torch.cuda.empty_cache()
+
+
 def run_report(args):
     import numpy as np
     import torch
@@ -702,6 +804,8 @@ def measure_extras(args, dec_inp, dev, stream, flush, world):
             "clocks": clk,
         }
         out[key]["roofline"]["traffic"] = recorded_traffic(f"grouped_ffn/{spec.name}")
+        if key == "prefill":
+            out[key]["overlap"] = time_overlap(spec, inp, dev, flush, args.steps, args.warmup)
         del inp, b
         torch.cuda.empty_cache()
     return out
@@ -820,7 +924,10 @@ def run_ours(args):
 
     extras = {}
     if args.config == "decode" and not overrides(args) and not args.no_extra:
-        extras = measure_extras(args, inp, dev, stream, flush, world)
+        # dispatch beside the grouped FFN on an SM partition (before the
+        # extras free the decode buffers' neighbours)
+        extras["overlap"] = time_overlap(spec, inp, dev, flush, args.steps, args.warmup)
+        extras.update(measure_extras(args, inp, dev, stream, flush, world))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -863,6 +970,8 @@ def main():
         run_reference(args)
     elif args.report:
         run_report(args)
+    elif args.overlap_sweep:
+        run_overlap_sweep(args)
     else:
         run_ours(args)
 

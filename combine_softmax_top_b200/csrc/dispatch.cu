@@ -394,7 +394,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   __shared__ uint32_t s_last;
   __shared__ uint32_t s_warp[kPlanThreads / 32];
   const int tid = threadIdx.x;
-  uint32_t* set = a.ws.set[a.ws.hdr->epoch_next & 1];
+  const uint32_t epoch = a.ws.hdr->epoch_next;
+  if (blockIdx.x == 0 && tid == 0) a.ws.hdr->epoch_plan = epoch;
+  uint32_t* set = a.ws.set[epoch & 1];
   uint32_t* pre = set_pre(set, a.E, a.tiles);
   uint32_t* base = set_base(set, a.E, a.tiles);
   for (int e = tid; e < a.E; e += kPlanThreads) hist[e] = 0u;
@@ -438,8 +440,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
 
 }  // namespace
 
+cudaError_t launch_plan(const Ctx& c, const int32_t* idx) {
+  PlanArgs pa;
+  pa.idx = idx;
+  pa.pairs = c.s.T * c.s.topk;
+  pa.E = (int)c.s.E;
+  pa.tiles = c.L.tiles;
+  pa.ws = c.ws;
+  const int64_t want = (pa.pairs + 8 * kPlanThreads - 1) / (8 * kPlanThreads);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, c.num_sms));
+  plan_kernel<<<grid, kPlanThreads, (size_t)pa.E * 4, c.stream>>>(pa);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
-                            const moe_dispatch_bufs& b, bool write_sf) {
+                            const moe_dispatch_bufs& b, bool write_sf, bool planned) {
   Args a;
   a.x = x;
   a.idx = idx;
@@ -457,21 +472,13 @@ cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
   a.ws = c.ws;
   a.xsf = write_sf && c.s.xq_dtype == MOE_E4M3 ? c.ws.xsf : nullptr;
   a.set_words = (int64_t)c.L.set_words;
-  if (a.compact) {
-    PlanArgs pa;
-    pa.idx = idx;
-    pa.pairs = (int64_t)a.T * a.k;
-    pa.E = a.E;
-    pa.tiles = a.tiles;
-    pa.ws = a.ws;
-    const int64_t want = (pa.pairs + 8 * kPlanThreads - 1) / (8 * kPlanThreads);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, c.num_sms));
-    plan_kernel<<<grid, kPlanThreads, (size_t)a.E * 4, c.stream>>>(pa);
-    const cudaError_t err = cudaGetLastError();
+  if (a.compact && !planned) {
+    const cudaError_t err = launch_plan(c, idx);
     if (err != cudaSuccess) return err;
   }
-  // one wave of resident CTAs, each walking several tokens (fewer CTAs also
-  // means fewer arrivals on the closing counter). The occupancy query is
+  // one wave of resident CTAs on the SMs given (all, or a partition's),
+  // each walking several tokens (fewer CTAs also means fewer arrivals on the
+  // closing counter). The occupancy query is
   // cached per device and kernel; concurrent callers may both run it, and
   // they store the same value.
   auto go = [&](auto kern, std::atomic<int>* cache) {

@@ -269,25 +269,86 @@ moe_status moe_layer_workspace_bytes(const moe_shape* shape, size_t* bytes) {
   return MOE_OK;
 }
 
+namespace moe {
+namespace {
+
+// The layer's intermediates inside a workspace of moe_layer_workspace_bytes.
+struct LayerPtrs {
+  moe_dispatch_bufs bufs;
+  int32_t* idx;
+  float* w;
+  void* y;
+};
+
+LayerPtrs layer_ptrs(const Ctx& c, void* ws) {
+  const LayerState ls = layer_state(c.s, c.L);
+  char* b = (char*)ws;
+  LayerPtrs lp;
+  lp.bufs.xq = b + ls.off_xq;
+  lp.bufs.xs = c.s.xq_dtype == MOE_E4M3 ? (float*)(b + ls.off_xs) : nullptr;
+  lp.bufs.counts = (int32_t*)(b + ls.off_counts);
+  lp.bufs.offsets = (int32_t*)(b + ls.off_offsets);
+  lp.bufs.row_src = (int32_t*)(b + ls.off_row_src);
+  lp.bufs.pos = (int32_t*)(b + ls.off_pos);
+  lp.bufs.hq = c.s.identity_experts ? nullptr : (void*)(b + ls.off_hq);
+  lp.bufs.hs = (!c.s.identity_experts && c.s.h_dtype == MOE_E4M3) ? (float*)(b + ls.off_hs) : nullptr;
+  lp.idx = (int32_t*)(b + ls.off_idx);
+  lp.w = (float*)(b + ls.off_w);
+  lp.y = c.s.identity_experts ? nullptr : (void*)(b + ls.off_y);
+  return lp;
+}
+
+}  // namespace
+}  // namespace moe
+
 moe_status moe_layer(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,
                      void* ws, void* out, moe_stream_t stream) {
   Ctx c;
   moe_status st = make_ctx(shape, ws, stream, &c);
   if (st != MOE_OK) return st;
-  const LayerState ls = layer_state(c.s, c.L);
-  char* b = (char*)ws;
-  moe_dispatch_bufs bufs;
-  bufs.xq = b + ls.off_xq;
-  bufs.xs = c.s.xq_dtype == MOE_E4M3 ? (float*)(b + ls.off_xs) : nullptr;
-  bufs.counts = (int32_t*)(b + ls.off_counts);
-  bufs.offsets = (int32_t*)(b + ls.off_offsets);
-  bufs.row_src = (int32_t*)(b + ls.off_row_src);
-  bufs.pos = (int32_t*)(b + ls.off_pos);
-  bufs.hq = c.s.identity_experts ? nullptr : (void*)(b + ls.off_hq);
-  bufs.hs = (!c.s.identity_experts && c.s.h_dtype == MOE_E4M3) ? (float*)(b + ls.off_hs) : nullptr;
-  void* y = c.s.identity_experts ? nullptr : (void*)(b + ls.off_y);
-  return moe_layer_bufs(shape, x, logits, w, (int32_t*)(b + ls.off_idx), (float*)(b + ls.off_w), &bufs, y, ws,
-                        out, stream);
+  LayerPtrs lp = layer_ptrs(c, ws);
+  return moe_layer_bufs(shape, x, logits, w, lp.idx, lp.w, &lp.bufs, lp.y, ws, out, stream);
+}
+
+moe_status moe_layer_overlap(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,
+                             void* ws, void* out, moe_stream_t stream, const moe_overlap* ov) {
+  // the shape and the partition arguments are checked before any CUDA call
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!ov || !ov->dispatch_stream || !ov->fork_event || !ov->join_event || ov->dispatch_stream == stream ||
+      ov->dispatch_sms < 1 || ov->ffn_sms < 0)
+    return MOE_ERR_INVALID_ARG;
+  Ctx c;
+  if ((st = make_ctx(shape, ws, stream, &c)) != MOE_OK) return st;
+  const int dsms = ov->dispatch_sms;
+  const int fsms = ov->ffn_sms ? ov->ffn_sms : c.num_sms - dsms;
+  if (dsms < 1 || dsms >= c.num_sms || fsms < 1 || fsms > c.num_sms - dsms) return MOE_ERR_INVALID_ARG;
+  if (!ffn_tc_supported(c.s)) return MOE_ERR_UNSUPPORTED;
+  LayerPtrs lp = layer_ptrs(c, ws);
+  // every argument is checked before the first launch
+  if (!tok_ok(c, logits) || !aligned16(logits) || !tok_ok(c, x) || !aligned16(x) || !tok_ok(c, out) ||
+      !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_weights(&c.s, w)) != MOE_OK) return st;
+  cudaEvent_t fork = (cudaEvent_t)ov->fork_event, join = (cudaEvent_t)ov->join_event;
+  if ((st = do_route(c, logits, lp.idx, lp.w)) != MOE_OK) return st;
+  if ((st = cuda_status(launch_plan(c, lp.idx))) != MOE_OK) return st;
+  if (cudaEventRecord(fork, c.stream) != cudaSuccess ||
+      cudaStreamWaitEvent((cudaStream_t)ov->dispatch_stream, fork, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // the FFN first, so that its persistent CTAs hold their SMs and dispatch
+  // takes the rest
+  Ctx cf = c;
+  cf.num_sms = fsms;
+  cf.streaming = true;
+  if ((st = cuda_status(launch_ffn_tc(cf, lp.bufs, *w, lp.y))) != MOE_OK) return st;
+  Ctx cd = c;
+  cd.num_sms = dsms;
+  cd.stream = (cudaStream_t)ov->dispatch_stream;
+  if ((st = cuda_status(launch_dispatch(cd, x, lp.idx, lp.bufs, true, true))) != MOE_OK) return st;
+  if (cudaEventRecord(join, cd.stream) != cudaSuccess || cudaStreamWaitEvent(c.stream, join, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return do_combine(c, &lp.bufs, lp.y, lp.w, out);
 }
 
 moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const float* logits, const moe_weights* w,

@@ -22,14 +22,17 @@ constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
 //
 // [header 256 B][counter set 0][counter set 1][sentinels][ring][xsf][hsf]
 //
-// header : epoch_next, epoch_cur, error, error_info (u32 each)
+// header : epoch_next, epoch_cur, error, error_info, epoch_plan (u32 each);
+//          epoch_plan is the epoch the counting pass planned, read by a grouped
+//          FFN that runs beside its dispatch (before epoch_cur moves on)
 // set    : misc[8] (ring_head, done, ring_total, ...) | count[E] |
 //          fill[tiles] | hdone[tiles] | pre[E] | base[E + 1]
 //          two sets are used alternately by consecutive dispatches; each
 //          dispatch zeroes the set the following dispatch will use.
 //          hdone[g] counts the finished gate/up slices of global tile g;
-//          pre / base: compact windows only (expert pair counts taken before
-//          dispatch, and each expert's first global tile).
+//          pre / base: the counting pass's expert pair counts, taken before
+//          dispatch (compact windows, or a grouped FFN run beside its
+//          dispatch), and each expert's first global tile (compact windows).
 // A global tile g covers rows 128 g .. 128 g + 127 of the expert buffers:
 // expert e's tile i is g = e * tpe + i (windows of cap rows) or base[e] + i
 // (compact windows); tiles = E * tpe or the compact bound.
@@ -44,7 +47,8 @@ struct Header {
   uint32_t epoch_cur;
   uint32_t error;
   uint32_t error_info;
-  uint32_t pad[60];
+  uint32_t epoch_plan;
+  uint32_t pad[59];
 };
 static_assert(sizeof(Header) == 256, "header size");
 
@@ -249,13 +253,20 @@ struct Ctx {
   Layout L;
   Ws ws;
   cudaStream_t stream;
-  int num_sms;
+  int num_sms;          // grid of the persistent kernels (all SMs, or a partition's share)
+  bool streaming = false;   // grouped FFN launched beside its dispatch (counts from the counting pass)
 };
 
 cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float* w);
-// write_sf: also write the e4m3 scale atoms the tensor-core FFN reads
+// write_sf: also write the e4m3 scale atoms the tensor-core FFN reads;
+// planned: the counting pass already ran (launch_plan), else compact windows
+// run it first
 cudaError_t launch_dispatch(const Ctx& c, const void* x, const int32_t* idx,
-                            const moe_dispatch_bufs& b, bool write_sf = true);
+                            const moe_dispatch_bufs& b, bool write_sf = true, bool planned = false);
+// The counting pass: per-expert pair counts (and, with compact windows, the
+// window layout) into the counter set of the next dispatch, and that
+// dispatch's epoch into Header::epoch_plan.
+cudaError_t launch_plan(const Ctx& c, const int32_t* idx);
 // The shared-memory-staged combine for many-token layers; false when the
 // shape does not suit it (nothing launched), else *err holds the launch result.
 bool launch_combine_tma(const Ctx& c, const moe_dispatch_bufs& b, const void* y, const float* topk_w, void* out,

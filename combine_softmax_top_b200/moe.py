@@ -26,7 +26,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 
 EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
            "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_layer_bufs", "moe_layer_workspace_bytes",
-           "moe_poll_status", "moe_status_string", "moe_dispatch_noalloc", "moe_pack_mx_scales")
+           "moe_poll_status", "moe_status_string", "moe_dispatch_noalloc", "moe_pack_mx_scales",
+           "moe_layer_overlap")
 
 
 class MoeError(RuntimeError):
@@ -54,6 +55,12 @@ class moe_dispatch_bufs(ctypes.Structure):
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")]
+
+
+class moe_overlap(ctypes.Structure):
+    _fields_ = [("dispatch_stream", ctypes.c_void_p), ("fork_event", ctypes.c_void_p),
+                ("join_event", ctypes.c_void_p), ("dispatch_sms", ctypes.c_int32),
+                ("ffn_sms", ctypes.c_int32)]
 
 
 _lib = None
@@ -85,6 +92,8 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch_noalloc": [S, P, P, ctypes.POINTER(moe_dispatch_bufs), P],
             "moe_status_string": [ctypes.c_int],
             "moe_pack_mx_scales": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P],
+            "moe_layer_overlap": [S, P, P, ctypes.POINTER(moe_weights), P, P, P,
+                                  ctypes.POINTER(moe_overlap)],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -180,6 +189,13 @@ def moe_layer_bufs(shape, x, logits, w: moe_weights, topk_idx, topk_w, bufs: moe
                                                   ctypes.byref(w), _ptr(topk_idx), _ptr(topk_w),
                                                   ctypes.byref(bufs), _ptr(y), _ptr(ws), _ptr(out),
                                                   _stream(stream)))
+
+
+def moe_layer_overlap(shape, x, logits, w: moe_weights, ws, out, ov: moe_overlap, stream=None) -> None:
+    """moe_layer with dispatch on ov.dispatch_stream beside the grouped FFN."""
+    _check("moe_layer_overlap", lib().moe_layer_overlap(ctypes.byref(shape), _ptr(x), _ptr(logits),
+                                                        ctypes.byref(w), _ptr(ws), _ptr(out), _stream(stream),
+                                                        ctypes.byref(ov)))
 
 
 def moe_pack_mx_scales(src: torch.Tensor, stream=None) -> torch.Tensor:
@@ -308,6 +324,48 @@ def run_layer_ws(lw: LayerWorkspace, inp: dict, stream=None) -> None:
     """Enqueue one whole layer (moe_layer, intermediates in the workspace)."""
     w = weights_struct(inp) if not lw.spec.identity else moe_weights()
     moe_layer(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, stream)
+
+
+class Overlap:
+    """A dispatch stream and the fork/join events moe_layer_overlap orders it
+    with (torch objects; the library only borrows their handles). With
+    green=True the dispatch stream belongs to a green context of
+    dispatch_sms SMs (torch.cuda.GreenContext), so the partition is enforced
+    by the device; otherwise the grouped FFN's grid leaves those SMs free."""
+
+    def __init__(self, dispatch_sms: int, ffn_sms: int = 0, green: bool = False, device=None):
+        self.green_ctx = None
+        if device is None:
+            index = torch.cuda.current_device()
+        elif isinstance(device, int):
+            index = device
+        else:
+            index = torch.device(device).index or 0
+        if green:
+            self.green_ctx = torch.cuda.GreenContext.create(int(dispatch_sms), int(index))
+            self._green_stream = self.green_ctx.Stream()
+            self.stream = torch.cuda.ExternalStream(self._green_stream.native_handle)
+        else:
+            # a high-priority stream: dispatch is the producer the FFN waits on
+            # (and high-priority streams never double as graph-capture streams)
+            self.stream = torch.cuda.Stream(device=index, priority=-1)
+        self.fork = torch.cuda.Event()
+        self.join = torch.cuda.Event()
+        # events exist once recorded: record both so their handles are real
+        self.fork.record(self.stream)
+        self.join.record(self.stream)
+        torch.cuda.synchronize(index)
+        self.ov = moe_overlap()
+        self.ov.dispatch_stream = self.stream.cuda_stream
+        self.ov.fork_event = self.fork.cuda_event
+        self.ov.join_event = self.join.cuda_event
+        self.ov.dispatch_sms = dispatch_sms
+        self.ov.ffn_sms = ffn_sms
+
+
+def run_layer_overlap(lw: "LayerWorkspace", inp: dict, ov: Overlap, stream=None) -> None:
+    """Enqueue one whole layer with dispatch beside the grouped FFN."""
+    moe_layer_overlap(lw.shape, inp["x"], inp["logits"], weights_struct(inp), lw.ws, lw.out, ov.ov, stream)
 
 
 # kernels the library launches per stage (mirrors the launch plan in csrc/)

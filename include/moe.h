@@ -312,6 +312,50 @@ MOE_API moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const f
                      moe_stream_t stream);
 
 /*
+ * How moe_layer_overlap splits the device between dispatch and the grouped
+ * FFN (all caller-owned; the library creates no stream or event).
+ *   dispatch_stream  a second stream, not the legacy default stream, that
+ *                    the dispatch kernel runs on; with a green context of
+ *                    dispatch_sms SMs (torch.cuda.GreenContext) its SMs are
+ *                    the partition's, else the SMs the grouped FFN leaves
+ *   fork_event       cudaEvent_t (cudaEventDisableTiming is enough):
+ *   join_event       recorded on `stream` / dispatch_stream to order the two
+ *   dispatch_sms     SMs dispatch is sized for: its grid is one wave of
+ *                    resident CTAs on that many SMs, 1 .. SMs - 1
+ *   ffn_sms          the grouped FFN's persistent grid (one CTA per SM);
+ *                    0 = the device's SMs minus dispatch_sms
+ */
+typedef struct moe_overlap {
+  moe_stream_t dispatch_stream;
+  void* fork_event;
+  void* join_event;
+  int32_t dispatch_sms;
+  int32_t ffn_sms;
+} moe_overlap;
+
+/*
+ * moe_layer with dispatch and the grouped FFN running at the same time on
+ * two parts of the device (GC-MoE explainer, "GC-MoE's Core Idea": a small
+ * partition of SMs dispatches while the rest computes; "Three-Node CUDA Graph
+ * and token-ring Handshake": the two kernels are concurrent, and the GEMM
+ * starts on the first filled tiles). On `stream`: route, then the counting
+ * pass (per-expert pair counts, and the compact window layout), then the
+ * grouped FFN on ffn_sms SMs, which takes its unit table from those counts
+ * and starts each tile once dispatch has published its sentinel; on
+ * dispatch_stream, between the fork and join events: dispatch; on `stream`
+ * after the join: combine. The result equals moe_layer's bit for bit.
+ *   arguments as moe_layer (ws of moe_layer_workspace_bytes, prepared by
+ *   moe_workspace_init), plus `ov`
+ * MOE_ERR_UNSUPPORTED for layers the tensor-core FFN does not run (fp32
+ * expert rows, identity experts); MOE_ERR_INVALID_ARG for a missing stream or
+ * event or SM counts out of range. A dispatch that never publishes a tile
+ * the FFN waits for ends in MOE_ERR_TIMEOUT (bounded waits), not a hang.
+ */
+MOE_API moe_status moe_layer_overlap(const moe_shape* shape, const void* x, const float* logits,
+                     const moe_weights* w, void* ws, void* out, moe_stream_t stream,
+                     const moe_overlap* ov);
+
+/*
  * moe_dispatch without a workspace argument, for callers that may not
  * allocate device memory where they dispatch (an engine that hands all device
  * memory to its own pool at start-up and forbids cudaMalloc while serving, or

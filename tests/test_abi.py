@@ -181,3 +181,33 @@ def test_layer_checks_arguments_before_any_launch():
     n = ctypes.c_size_t(0)
     assert L.moe_layer_workspace_bytes(ctypes.byref(bad), ctypes.byref(n)) == 1
     assert L.moe_layer_workspace_bytes(ctypes.byref(sh), None) == 1
+
+
+def test_overlap_checks_its_partition_before_any_cuda_call():
+    """moe_layer_overlap refuses a missing overlap description, a missing
+    stream or event, the dispatch stream equal to the layer's stream, and an
+    empty dispatch partition, all on the host."""
+    sh = moe.make_shape(W.spec("decode"))
+    L = moe.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    w = moe.moe_weights()
+    assert L.moe_layer_overlap(ctypes.byref(sh), fake, fake, ctypes.byref(w), fake, fake, None, None) == 1
+
+    def ov(**kw):
+        o = moe.moe_overlap()
+        o.dispatch_stream, o.fork_event, o.join_event, o.dispatch_sms, o.ffn_sms = 1 << 12, 1 << 13, 1 << 14, 20, 0
+        for k, v in kw.items():
+            setattr(o, k, v)
+        return o
+
+    for bad in (dict(dispatch_stream=0), dict(fork_event=0), dict(join_event=0), dict(dispatch_sms=0),
+                dict(dispatch_sms=-3), dict(ffn_sms=-1), dict(dispatch_stream=1 << 16)):
+        o = ov(**bad)
+        stream = ctypes.c_void_p(1 << 16)       # the last case: the same stream twice
+        assert L.moe_layer_overlap(ctypes.byref(sh), fake, fake, ctypes.byref(w), fake, fake, stream,
+                                   ctypes.byref(o)) == 1, bad
+    bad = moe.make_shape(W.spec("decode"))
+    bad.topk = 0
+    o = ov()
+    assert L.moe_layer_overlap(ctypes.byref(bad), fake, fake, ctypes.byref(w), fake, fake, None,
+                               ctypes.byref(o)) == 1
