@@ -54,10 +54,11 @@ constexpr int kTailMax = 32;
 
 // Shared-memory stage for a variant whose token tiles hold up to kBRows rows:
 // A0 | A1 | B (kBRows (+ kTailMax) x 128 B, or two slabs of N rows) | SFA0 |
-// SFA1 | SFB0 | SFB1 (the joined tail's token scales)
-template <int kBRows>
+// SFA1 | SFB0 | SFB1 (the joined tail's token scales). With kPair = 2 (a CTA
+// pair sharing each MMA) every CTA holds half of the token rows.
+template <int kBRows, int kPair = 1>
 struct Stage {
-  static constexpr int kBRowsMax = kBRows + (kBRows > 64 ? kTailMax : 0);
+  static constexpr int kBRowsMax = (kBRows + (kBRows > 64 ? kTailMax : 0)) / kPair;
   static constexpr int kOffA1 = kABytes;
   static constexpr int kOffB = 2 * kABytes;
   static constexpr int kOffSfa0 = kOffB + kBRowsMax * kSlab;
@@ -90,6 +91,7 @@ enum : int { kFfnGen = 3, kFfnExit = 4, kFfnNext = 5 };
 struct TcParams {
   CUtensorMap tm_wg, tm_wu, tm_wd;
   CUtensorMap tm_x[4], tm_h[4];   // token rows in boxes of 16, 32, 64, 128 rows
+  CUtensorMap tm_xsf, tm_hsf;     // CTA pairs: token scale atoms as rows of 128 words (one atom per box)
   const void* sg;   // weight scales: fp32 per 128 x 128 block (e4m3) or UE8M0 atoms (e2m1)
   const void* su;
   const void* sd;
@@ -99,6 +101,8 @@ struct TcParams {
   Ws ws;
   int H, I, E, cap, tpe;
   int compact;               // expert windows start at base[e] tiles (set_base)
+  int streaming;             // launched beside its dispatch: the counting pass's epoch and
+                             // counts, no closed tile total
   int n_islices, n_hslices;  // I/128, H/128
   int nk1, nk2;              // K slabs of gate/up (over H) and down (over I)
   int kelems;                // elements per slab
@@ -144,12 +148,21 @@ __device__ __forceinline__ int4 shfl_int4(int4 v) {
 }
 
 // Bounded wait on an mbarrier phase; false on timeout (latched) or abort.
+// kCl: the phase includes arrivals from the other CTA of a pair, whose writes
+// the waiter then sees (acquire at cluster scope).
+template <bool kCl = false>
+__device__ __forceinline__ bool try_bar(uint64_t* bar, uint32_t parity) {
+  if constexpr (kCl) return ptx::mbar_try_wait_cluster(bar, parity);
+  else return ptx::mbar_try_wait(bar, parity);
+}
+
+template <bool kCl = false>
 __device__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, Header* hdr,
                          uint32_t where) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (try_bar<kCl>(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (try_bar<kCl>(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitBudgetNs) {
       latch_error(hdr, MOE_ERR_TIMEOUT, where);
@@ -267,10 +280,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const uint32_t epoch = p.ws.hdr->epoch_cur;
+  // Beside its dispatch (streaming), the epoch is the one the counting pass
+  // planned and the per-expert counts are its counts; tiles are taken as
+  // their sentinels appear, before the dispatch has closed. After the
+  // dispatch, the epoch it closed and its final counts and tile total.
+  const uint32_t epoch = p.streaming ? p.ws.hdr->epoch_plan : p.ws.hdr->epoch_cur;
   uint32_t* set = p.ws.set[epoch & 1];
   uint32_t* misc = set_misc(set);
-  const uint32_t ntiles = ld_acquire(misc + kRingTotal);
+  const uint32_t ntiles = p.streaming ? 0u : ld_acquire(misc + kRingTotal);
   const uint32_t gen = ld_acquire(misc + kFfnGen);   // FFN calls already made on this dispatch
   uint32_t* hdone = set_hdone(set, p.E, p.tiles);
   // down units cover two slices of H each when tiles are large (the two share
@@ -306,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     const uint32_t* base = p.compact ? set_base(set, p.E, p.tiles) : nullptr;
     int ntab = 0;   // tiles counted from the expert counts (lane 31)
     {
-      const uint32_t* cnt = set_count(set);
+      const uint32_t* cnt = p.streaming ? set_pre(set, p.E, p.tiles) : set_count(set);
       const int per = (p.E + 31) / 32;
       auto tiles_of = [&](int e, int* tail) {
         const int c = (int)min(ld_acquire(cnt + e), (uint32_t)p.cap);
@@ -357,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         ++i;
         return true;
       };
-      if ((uint32_t)ntab != ntiles) {   // the published tile total disagrees with the counts
+      if (!p.streaming && (uint32_t)ntab != ntiles) {   // the published tile total disagrees with the counts
         latch_error(hdr, MOE_ERR_INVALID_ARG, 0x24000000u | (uint32_t)ntab);
         *abort_flag = 1;
         good = false;
@@ -1059,6 +1076,7 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.cap = (int)c.L.cap;
   p.tpe = (int)c.L.tpe;
   p.compact = c.L.compact ? 1 : 0;
+  p.streaming = c.streaming ? 1 : 0;
   p.n_islices = (int)(I / 128);
   p.n_hslices = (int)(H / 128);
   p.kelems = kel;
