@@ -103,6 +103,9 @@ struct TcParams {
   int compact;               // expert windows start at base[e] tiles (set_base)
   int streaming;             // launched beside its dispatch: the counting pass's epoch and
                              // counts, no closed tile total
+  int R;                     // windows per weight expert: 1, or the source ranks of expert
+                             // parallelism (virtual expert v uses the weights of v / R)
+  int ep_sources;            // expert parallelism: wait for this many closed sources (else 0)
   int n_islices, n_hslices;  // I/128, H/128
   int nk1, nk2;              // K slabs of gate/up (over H) and down (over I)
   int kelems;                // elements per slab
@@ -287,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
   const uint32_t epoch = p.streaming ? p.ws.hdr->epoch_plan : p.ws.hdr->epoch_cur;
   uint32_t* set = p.ws.set[epoch & 1];
   uint32_t* misc = set_misc(set);
-  const uint32_t ntiles = p.streaming ? 0u : ld_acquire(misc + kRingTotal);
+  const uint32_t ntiles_early = (p.streaming || p.ep_sources) ? 0u : ld_acquire(misc + kRingTotal);
   const uint32_t gen = ld_acquire(misc + kFfnGen);   // FFN calls already made on this dispatch
   uint32_t* hdone = set_hdone(set, p.E, p.tiles);
   // down units cover two slices of H each when tiles are large (the two share
@@ -320,6 +323,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
     // expert's last tile of at most kTailMax rows joins the tile before it:
     // its weights are then not streamed again for a few tokens.
     int* chunk_tab = reinterpret_cast<int*>(ctl + kCtlBytes);   // [E + 1]
+    if (p.ep_sources && lane == 0) {   // every source rank has closed its dispatch into these windows
+      const unsigned long long t0 = globaltimer();
+      uint32_t n;
+      while (true) {
+        asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(n) : "l"(misc + kSrcDone) : "memory");
+        if (n >= (uint32_t)p.ep_sources || *abort_flag) break;
+        if (globaltimer() - t0 > kWaitBudgetNs) {
+          latch_error(hdr, MOE_ERR_TIMEOUT, 0x26000000u | n);
+          *abort_flag = 1;
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    __syncwarp();
     const uint32_t* base = p.compact ? set_base(set, p.E, p.tiles) : nullptr;
     int ntab = 0;   // tiles counted from the expert counts (lane 31)
     {
@@ -363,6 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       ntab = __shfl_sync(0xffffffffu, it, 31);
       __syncwarp();
     }
+    // (with expert parallelism the sources' tile totals are complete only now)
+    const uint32_t ntiles = p.ep_sources ? ld_acquire(misc + kRingTotal) : ntiles_early;
     if (lane == 0) {
       uint32_t i = 0;
       bool good = true;
@@ -391,24 +411,32 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         j.kind = u >= n1 ? kKindDown : kKindGateUp;
         const uint32_t v = j.kind == kKindDown ? u - n1 : u;
         const uint32_t ns = (uint32_t)(j.kind == kKindDown ? p.n_hslices / dpair : p.n_islices);
-        // expert: the last e with first_chunk[e] * ns <= v (empty experts never are)
-        int lo = 0, hi = p.E - 1;
+        // weight expert: the last we with first_chunk[we * R] * ns <= v (empty
+        // ones never are); its units cover the chunks of its R windows
+        // (consecutive in chunk_tab), slice-major, so that the windows sharing
+        // a weight slice are worked on together
+        const int R = p.R;
+        int lo = 0, hi = p.E / R - 1;
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
-          if ((uint32_t)(chunk_tab[mid] & 0xFFFFFF) * ns <= v) lo = mid;
+          if ((uint32_t)(chunk_tab[mid * R] & 0xFFFFFF) * ns <= v) lo = mid;
           else hi = mid - 1;
         }
-        j.e = lo;
-        const int c0 = chunk_tab[lo] & 0xFFFFFF;
-        const int tail = (int)((uint32_t)chunk_tab[lo] >> 24);
-        const uint32_t nc = (uint32_t)((chunk_tab[lo + 1] & 0xFFFFFF) - c0);
+        const int c0 = chunk_tab[lo * R] & 0xFFFFFF;
+        const uint32_t nc = (uint32_t)((chunk_tab[(lo + 1) * R] & 0xFFFFFF) - c0);
         const uint32_t w = v - (uint32_t)c0 * ns;
+        const int cc = c0 + (int)(w % nc);   // the unit's chunk
+        int ve = lo * R;                      // its window: the last with first chunk <= cc
+        while (ve + 1 < (lo + 1) * R && (chunk_tab[ve + 1] & 0xFFFFFF) <= cc) ++ve;
+        j.e = ve;
+        const int tail = (int)((uint32_t)chunk_tab[ve] >> 24);
+        const int ncv = (chunk_tab[ve + 1] & 0xFFFFFF) - (chunk_tab[ve] & 0xFFFFFF);
         j.pair = j.kind == kKindDown && dpair == 2;
         j.slice = (int)(w / nc) * (j.pair ? 2 : 1);
-        j.tile = (int)(w % nc);
+        j.tile = cc - (chunk_tab[ve] & 0xFFFFFF);
         // global tile: rows 128 * slot ..., the down units' counter
         j.slot = (base ? (int)base[j.e] : j.e * p.tpe) + j.tile;
-        j.wide = tail && j.tile == (int)nc - 1;
+        j.wide = tail && j.tile == ncv - 1;
         int rows = 0;
         good = wait_tile(p, epoch, j.slot, abort_flag, &rows);
         if (good && j.wide) {   // the joined tail's sentinel too
@@ -468,7 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       const bool down = j.kind == kKindDown;
       const int N = (j.rows + 15) & ~15;
       const int nsteps = down ? p.nk2 / j.nslab : p.nk1;
-      const int arow = j.e * (down ? p.H : p.I) + j.slice * 128;
+      const int we = j.e / p.R;   // the window's weight expert
+      const int arow = we * (down ? p.H : p.I) + j.slice * 128;
       const int brow = j.slot * kTileRows + j.row_off;
       const int64_t tile_g = j.slot;
       const bool dual = !down || j.pair;   // two weight tiles share the token tile
@@ -483,19 +512,19 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
       uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
       int sbase = 0;   // first K block held in sa*/sb*
       const int nkb = down ? p.I / 128 : p.H / 128;
-      const float* pa = down ? (const float*)p.sd + ((int64_t)j.e * p.n_hslices + j.slice) * nkb
-                             : (const float*)p.sg + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
-      const float* pb = down ? (const float*)p.sd + ((int64_t)j.e * p.n_hslices + j.slice + 1) * nkb
-                             : (const float*)p.su + ((int64_t)j.e * p.n_islices + j.slice) * nkb;
+      const float* pa = down ? (const float*)p.sd + ((int64_t)we * p.n_hslices + j.slice) * nkb
+                             : (const float*)p.sg + ((int64_t)we * p.n_islices + j.slice) * nkb;
+      const float* pb = down ? (const float*)p.sd + ((int64_t)we * p.n_hslices + j.slice + 1) * nkb
+                             : (const float*)p.su + ((int64_t)we * p.n_islices + j.slice) * nkb;
       // 4-bit weights: the scale atoms of the job's weight tiles, one per
       // 128-value K block (row-major over [slice][K block])
       const uint8_t* atom_a = nullptr;
       const uint8_t* atom_b = nullptr;
       if constexpr (kW4) {
         const int n_out = down ? p.n_hslices : p.n_islices;
-        atom_a = (const uint8_t*)(down ? p.sd : p.sg) + ((int64_t)j.e * n_out + j.slice) * nkb * kSfAtomBytes;
+        atom_a = (const uint8_t*)(down ? p.sd : p.sg) + ((int64_t)we * n_out + j.slice) * nkb * kSfAtomBytes;
         atom_b = down ? atom_a + (int64_t)nkb * kSfAtomBytes
-                      : (const uint8_t*)p.su + ((int64_t)j.e * n_out + j.slice) * nkb * kSfAtomBytes;
+                      : (const uint8_t*)p.su + ((int64_t)we * n_out + j.slice) * nkb * kSfAtomBytes;
       }
       // A scale that is not a normal power of two latches
       // MOE_ERR_INVALID_ARG (info: 0x25, the matrix (0 gate / down, 1 up or
@@ -517,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tc_kernel(const __grid_consta
         }
         const uint32_t which = __ballot_sync(0xffffffffu, bad_a) ? 0u : 1u;
         if (__ballot_sync(0xffffffffu, bad) != 0u && lane == 0)
-          latch_error(hdr, MOE_ERR_INVALID_ARG, 0x25000000u | (which << 20) | (uint32_t)j.e);
+          latch_error(hdr, MOE_ERR_INVALID_ARG, 0x25000000u | (which << 20) | (uint32_t)we);
       };
       // the four exponents of blocks kr .. kr+3 (relative to sbase), packed
       auto pack4 = [&](uint32_t r0, uint32_t r1, int kr) -> uint32_t {
@@ -1077,6 +1106,8 @@ cudaError_t launch_typed(const Ctx& c, const moe_dispatch_bufs& b, const moe_wei
   p.tpe = (int)c.L.tpe;
   p.compact = c.L.compact ? 1 : 0;
   p.streaming = c.streaming ? 1 : 0;
+  p.R = c.ep_ranks > 0 ? c.ep_ranks : 1;
+  p.ep_sources = c.ep_ranks > 0 ? c.ep_ranks : 0;
   p.n_islices = (int)(I / 128);
   p.n_hslices = (int)(H / 128);
   p.kelems = kel;

@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/moe.h: argument checks, the
 // workspace, and the kernel launches of each stage.
+#include <algorithm>
 #include <cstring>
 
 #include "moe_internal.cuh"
@@ -372,6 +373,147 @@ moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const float* lo
   if ((st = do_dispatch(c, x, topk_idx, bufs)) != MOE_OK) return st;
   if ((st = do_ffn(c, bufs, w, y)) != MOE_OK) return st;
   return do_combine(c, bufs, y, topk_w, out);
+}
+
+// ---- expert parallelism ------------------------------------------------------
+
+namespace moe {
+namespace {
+
+// The global layer shape and the rank's place in it.
+moe_status check_ep(const moe_shape* s, const moe_ep* ep) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!ep || ep->ranks < 1 || ep->ranks > 64 || ep->rank < 0 || ep->rank >= ep->ranks || ep->reserved != 0 ||
+      (ep->protocol != MOE_EP_SENTINEL && ep->protocol != MOE_EP_FENCE) || ep->t_max < s->T || ep->t_max < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->E % ep->ranks != 0 || s->cap_rows != 0 || (s->flags & MOE_FLAG_COMPACT)) return MOE_ERR_INVALID_ARG;
+  if (s->flags & MOE_FLAG_SHARED_EXPERT) return MOE_ERR_UNSUPPORTED;
+  const EpGeom g = make_ep_geom(*s, *ep);
+  if ((st = check_shape(&g.rs)) != MOE_OK) return st;   // the receivers' windows
+  if ((int64_t)ep->ranks * g.rows >= (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;   // pos is int32
+  return MOE_OK;
+}
+
+moe_status ep_ctx(const moe_shape* s, const moe_ep* ep, const moe_ep_windows* all, moe_stream_t stream, Ctx* c,
+                  EpGeom* g) {
+  moe_status st = check_ep(s, ep);
+  if (st != MOE_OK) return st;
+  if (!all || !all->ws || ((uintptr_t)all->ws & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  *g = make_ep_geom(*s, *ep);
+  if ((st = make_ctx(s, (char*)all->ws + (size_t)ep->rank * g->ws_bytes, stream, c)) != MOE_OK) return st;
+  return MOE_OK;
+}
+
+size_t el_bytes(int32_t d) { return d == MOE_F32 ? 4 : (d == MOE_BF16 ? 2 : 1); }
+
+}  // namespace
+}  // namespace moe
+
+moe_status moe_ep_sizes(const moe_shape* shape, const moe_ep* ep, int64_t* rows, size_t* ws_bytes) {
+  moe_status st = check_ep(shape, ep);
+  if (st != MOE_OK) return st;
+  if (!rows || !ws_bytes) return MOE_ERR_INVALID_ARG;
+  const EpGeom g = make_ep_geom(*shape, *ep);
+  *rows = g.rows;
+  *ws_bytes = g.ws_bytes;
+  return MOE_OK;
+}
+
+moe_status moe_ep_workspace_init(const moe_shape* shape, const moe_ep* ep, const moe_ep_windows* all,
+                                 moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  const size_t words = g.ws_bytes / 4;
+  const int grid = (int)std::min<size_t>((words + 255) / 256, (size_t)c.num_sms * 8);
+  init_ws_kernel<<<grid > 0 ? grid : 1, 256, 0, c.stream>>>((uint32_t*)c.ws.hdr, words);
+  return cuda_status(cudaGetLastError());
+}
+
+moe_status moe_ep_count(const moe_shape* shape, const moe_ep* ep, const int32_t* topk_idx,
+                        const moe_ep_windows* all, moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  if (ep->protocol != MOE_EP_FENCE || !tok_ok(c, topk_idx)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_count(c, g, topk_idx, *all));
+}
+
+moe_status moe_ep_layout(const moe_shape* shape, const moe_ep* ep, const moe_ep_windows* all, moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  if (ep->protocol != MOE_EP_FENCE) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_layout(c, g, *all));
+}
+
+moe_status moe_ep_dispatch(const moe_shape* shape, const moe_ep* ep, const void* x, const int32_t* topk_idx,
+                           const moe_ep_windows* all, int32_t* pos, moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  if (!tok_ok(c, x) || !aligned16(x) || !tok_ok(c, topk_idx) || !tok_ok(c, pos)) return MOE_ERR_INVALID_ARG;
+  if (!all->xq || !aligned16(all->xq) || !all->row_src || (c.s.xq_dtype == MOE_E4M3 && !all->xs))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_dispatch(c, g, x, topk_idx, *all, pos));
+}
+
+moe_status moe_ep_grouped_ffn(const moe_shape* shape, const moe_ep* ep, const moe_weights* w,
+                              const moe_ep_windows* all, moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  if (shape->identity_experts) return MOE_OK;
+  if (!ffn_tc_supported(g.rs)) return MOE_ERR_UNSUPPORTED;   // the tensor-core FFN's formats
+  if ((st = check_weights(&g.rs, w)) != MOE_OK) return st;
+  if (!all->xq || !all->hq || !all->y || (g.rs.xq_dtype == MOE_E4M3 && !all->xs) ||
+      (g.rs.h_dtype == MOE_E4M3 && !all->hs))
+    return MOE_ERR_INVALID_ARG;
+  // this rank's part of the rank-major windows, as a receiver of V windows
+  const int64_t r0 = (int64_t)ep->rank * g.rows;
+  moe_dispatch_bufs b;
+  memset(&b, 0, sizeof(b));
+  b.xq = (char*)all->xq + r0 * g.rs.H * (int64_t)el_bytes(g.rs.xq_dtype);
+  b.xs = all->xs ? all->xs + r0 * (g.rs.H / kQBlock) : nullptr;
+  b.hq = (char*)all->hq + r0 * g.rs.I * (int64_t)el_bytes(g.rs.h_dtype);
+  b.hs = all->hs ? all->hs + r0 * (g.rs.I / kQBlock) : nullptr;
+  b.row_src = all->row_src ? all->row_src + r0 : nullptr;
+  void* y = (char*)all->y + r0 * g.rs.H * (int64_t)el_bytes(g.rs.y_dtype);
+  if (!aligned16(b.xq) || !aligned16(b.hq) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  Ctx cf = c;
+  cf.s = g.rs;
+  cf.L = g.RL;
+  cf.ws = ws_view(c.ws.hdr, g.RL);
+  cf.ep_ranks = g.R;
+  if ((st = cuda_status(launch_ffn_tc(cf, b, *w, y))) != MOE_OK) return st;
+  return cuda_status(launch_ep_publish_y(cf));
+}
+
+moe_status moe_ep_combine(const moe_shape* shape, const moe_ep* ep, const int32_t* pos, const float* topk_w,
+                          const moe_ep_windows* all, void* out, moe_stream_t stream) {
+  Ctx c;
+  EpGeom g;
+  moe_status st = ep_ctx(shape, ep, all, stream, &c, &g);
+  if (st != MOE_OK) return st;
+  if (!tok_ok(c, pos) || !tok_ok(c, topk_w) || !tok_ok(c, out) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  moe_dispatch_bufs b;
+  memset(&b, 0, sizeof(b));
+  b.pos = const_cast<int32_t*>(pos);
+  if (shape->identity_experts) {   // the pushed tokens are complete once this rank's dispatch is
+    if (!all->xq || !aligned16(all->xq) || (c.s.xq_dtype == MOE_E4M3 && !all->xs)) return MOE_ERR_INVALID_ARG;
+    b.xq = all->xq;
+    b.xs = all->xs;
+    return cuda_status(launch_combine(c, b, nullptr, topk_w, out));
+  }
+  if (!all->y || !aligned16(all->y)) return MOE_ERR_INVALID_ARG;
+  if ((st = cuda_status(launch_ep_wait_y(c, g, *all))) != MOE_OK) return st;
+  return cuda_status(launch_combine(c, b, all->y, topk_w, out));
 }
 
 moe_status moe_poll_status(void* ws, moe_stream_t stream) {

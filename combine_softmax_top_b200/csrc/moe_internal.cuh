@@ -22,9 +22,11 @@ constexpr unsigned long long kWaitBudgetNs = 200ull * 1000ull * 1000ull;
 //
 // [header 256 B][counter set 0][counter set 1][sentinels][ring][xsf][hsf]
 //
-// header : epoch_next, epoch_cur, error, error_info, epoch_plan (u32 each);
-//          epoch_plan is the epoch the counting pass planned, read by a grouped
-//          FFN that runs beside its dispatch (before epoch_cur moves on)
+// header : epoch_next, epoch_cur, error, error_info, epoch_plan, layout_ready,
+//          y_ready (u32 each); epoch_plan is the epoch the counting pass
+//          planned, read by a grouped FFN that runs beside its dispatch (before
+//          epoch_cur moves on); layout_ready / y_ready are the expert-parallel
+//          flags other ranks poll
 // set    : misc[8] (ring_head, done, ring_total, ...) | count[E] |
 //          fill[tiles] | hdone[tiles] | pre[E] | base[E + 1]
 //          two sets are used alternately by consecutive dispatches; each
@@ -48,11 +50,17 @@ struct Header {
   uint32_t error;
   uint32_t error_info;
   uint32_t epoch_plan;
-  uint32_t pad[59];
+  uint32_t layout_ready;   // expert parallelism, Fence: epoch whose window layout is laid out here
+  uint32_t y_ready;        // expert parallelism: epoch whose expert outputs y are complete here
+  uint32_t pad[57];
 };
 static_assert(sizeof(Header) == 256, "header size");
 
-enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kPlanDone = 6, kMiscWords = 8 };
+// misc slots of a counter set (3-5 belong to the grouped FFN); kSrcDone and
+// kSrcCounted count the source ranks that closed their dispatch into this
+// rank's windows / wrote their pair counts here (expert parallelism)
+enum MiscSlot { kRingHead = 0, kDone = 1, kRingTotal = 2, kPlanDone = 6, kSrcDone = 8, kSrcCounted = 9,
+                kMiscWords = 16 };
 
 struct Layout {
   int64_t T, H, E, k, I, cap, tpe, tiles;   // tiles: E * tpe, or the compact bound
@@ -255,7 +263,58 @@ struct Ctx {
   cudaStream_t stream;
   int num_sms;          // grid of the persistent kernels (all SMs, or a partition's share)
   bool streaming = false;   // grouped FFN launched beside its dispatch (counts from the counting pass)
+  int ep_ranks = 0;     // grouped FFN of one rank under expert parallelism: windows of
+                        // E_loc * R regions (one per local expert and source rank), R closes awaited
 };
+
+// ---- expert parallelism (ep.cu) ----------------------------------------------
+//
+// R ranks, rank d owning experts [d E_loc, (d + 1) E_loc), E_loc = E / R.
+// Every rank receives into windows of V = E virtual experts, v = el * R + src
+// (local expert el, source rank src): rank-major regions per source inside
+// each expert's block, so that each source fills its own regions without
+// asking anyone where (no metadata exchanged first). Sentinel protocol:
+// regions of cap_src = round_up(t_max, 128) rows. Fence protocol: every
+// source's pair counts are written to the receivers first, each receiver lays
+// its regions out back to back in whole tiles (as compact windows), and
+// sources place rows at exact offsets. All ranks' windows and workspaces are
+// reached through rank-major address ranges (rank d's part at d * stride).
+struct EpGeom {
+  int R, rank, e_loc, protocol;
+  int64_t t_max, cap_src, tpe_src, rows;   // rows of one rank's windows
+  moe_shape rs;          // the receiver's shape: E = V virtual experts
+  Layout RL;             // the receiver's workspace layout
+  size_t src_off;        // the source's claim counters: [2][E + 8] u32 after RL.total
+  size_t ws_bytes;       // one rank's workspace
+};
+
+inline EpGeom make_ep_geom(const moe_shape& s, const moe_ep& ep) {
+  EpGeom g{};
+  g.R = ep.ranks;
+  g.rank = ep.rank;
+  g.e_loc = (int)(s.E / ep.ranks);
+  g.protocol = ep.protocol;
+  g.t_max = ep.t_max;
+  g.rs = s;
+  g.rs.E = s.E;                                   // V = E_loc * R = E
+  if (ep.protocol == MOE_EP_FENCE) {
+    g.rs.flags = MOE_FLAG_COMPACT;
+    g.rs.T = ep.t_max * ep.ranks;
+    g.rs.topk = s.topk < g.e_loc ? s.topk : g.e_loc;   // pairs one token sends one rank
+    g.rs.cap_rows = 0;
+  } else {
+    g.rs.flags = 0;
+    g.rs.T = ep.t_max;
+    g.rs.cap_rows = ceil_div(ep.t_max > 0 ? ep.t_max : 1, kTileRows) * kTileRows;
+  }
+  g.RL = make_layout(g.rs);
+  g.cap_src = g.RL.cap;
+  g.tpe_src = g.RL.tpe;
+  g.rows = g.RL.tiles * kTileRows;
+  g.src_off = align_up(g.RL.total, 256);
+  g.ws_bytes = align_up(g.src_off + 2 * (size_t)(s.E + 8) * 4, 256);
+  return g;
+}
 
 cudaError_t launch_route(const Ctx& c, const float* logits, int32_t* idx, float* w);
 // write_sf: also write the e4m3 scale atoms the tensor-core FFN reads;
@@ -278,5 +337,13 @@ cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_
 cudaError_t launch_ffn_tc(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,
                           void* y);
 bool ffn_tc_supported(const moe_shape& s);
+
+// expert parallelism (ep.cu); g describes this rank, `all` the rank-major ranges
+cudaError_t launch_ep_count(const Ctx& c, const EpGeom& g, const int32_t* idx, const moe_ep_windows& all);
+cudaError_t launch_ep_layout(const Ctx& c, const EpGeom& g, const moe_ep_windows& all);
+cudaError_t launch_ep_dispatch(const Ctx& c, const EpGeom& g, const void* x, const int32_t* idx,
+                               const moe_ep_windows& all, int32_t* pos);
+cudaError_t launch_ep_publish_y(const Ctx& c);
+cudaError_t launch_ep_wait_y(const Ctx& c, const EpGeom& g, const moe_ep_windows& all);
 
 }  // namespace moe

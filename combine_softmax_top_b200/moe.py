@@ -27,7 +27,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_workspace_bytes", "moe_workspace_init", "moe_route", "moe_dispatch",
            "moe_grouped_ffn", "moe_combine", "moe_layer", "moe_layer_bufs", "moe_layer_workspace_bytes",
            "moe_poll_status", "moe_status_string", "moe_dispatch_noalloc", "moe_pack_mx_scales",
-           "moe_layer_overlap")
+           "moe_layer_overlap", "moe_ep_sizes", "moe_ep_workspace_init", "moe_ep_count", "moe_ep_layout",
+           "moe_ep_dispatch", "moe_ep_grouped_ffn", "moe_ep_combine")
 
 
 class MoeError(RuntimeError):
@@ -63,6 +64,18 @@ class moe_overlap(ctypes.Structure):
                 ("ffn_sms", ctypes.c_int32)]
 
 
+MOE_EP_SENTINEL, MOE_EP_FENCE = 0, 1
+
+
+class moe_ep(ctypes.Structure):
+    _fields_ = [("ranks", ctypes.c_int32), ("rank", ctypes.c_int32), ("protocol", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("t_max", ctypes.c_int64)]
+
+
+class moe_ep_windows(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("xq", "xs", "row_src", "hq", "hs", "y", "ws")]
+
+
 _lib = None
 
 
@@ -94,6 +107,15 @@ def lib() -> ctypes.CDLL:
             "moe_pack_mx_scales": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P],
             "moe_layer_overlap": [S, P, P, ctypes.POINTER(moe_weights), P, P, P,
                                   ctypes.POINTER(moe_overlap)],
+            "moe_ep_sizes": [S, ctypes.POINTER(moe_ep), ctypes.POINTER(ctypes.c_int64),
+                             ctypes.POINTER(ctypes.c_size_t)],
+            "moe_ep_workspace_init": [S, ctypes.POINTER(moe_ep), ctypes.POINTER(moe_ep_windows), P],
+            "moe_ep_count": [S, ctypes.POINTER(moe_ep), P, ctypes.POINTER(moe_ep_windows), P],
+            "moe_ep_layout": [S, ctypes.POINTER(moe_ep), ctypes.POINTER(moe_ep_windows), P],
+            "moe_ep_dispatch": [S, ctypes.POINTER(moe_ep), P, P, ctypes.POINTER(moe_ep_windows), P, P],
+            "moe_ep_grouped_ffn": [S, ctypes.POINTER(moe_ep), ctypes.POINTER(moe_weights),
+                                   ctypes.POINTER(moe_ep_windows), P],
+            "moe_ep_combine": [S, ctypes.POINTER(moe_ep), P, P, ctypes.POINTER(moe_ep_windows), P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -196,6 +218,45 @@ def moe_layer_overlap(shape, x, logits, w: moe_weights, ws, out, ov: moe_overlap
     _check("moe_layer_overlap", lib().moe_layer_overlap(ctypes.byref(shape), _ptr(x), _ptr(logits),
                                                         ctypes.byref(w), _ptr(ws), _ptr(out), _stream(stream),
                                                         ctypes.byref(ov)))
+
+
+def moe_ep_sizes(shape, ep: moe_ep) -> tuple[int, int]:
+    """(rows of one rank's windows, bytes of one rank's workspace)."""
+    rows, nb = ctypes.c_int64(0), ctypes.c_size_t(0)
+    _check("moe_ep_sizes", lib().moe_ep_sizes(ctypes.byref(shape), ctypes.byref(ep), ctypes.byref(rows),
+                                              ctypes.byref(nb)))
+    return rows.value, nb.value
+
+
+def moe_ep_workspace_init(shape, ep: moe_ep, win: moe_ep_windows, stream=None) -> None:
+    _check("moe_ep_workspace_init", lib().moe_ep_workspace_init(ctypes.byref(shape), ctypes.byref(ep),
+                                                                ctypes.byref(win), _stream(stream)))
+
+
+def moe_ep_count(shape, ep: moe_ep, topk_idx, win: moe_ep_windows, stream=None) -> None:
+    _check("moe_ep_count", lib().moe_ep_count(ctypes.byref(shape), ctypes.byref(ep), _ptr(topk_idx),
+                                              ctypes.byref(win), _stream(stream)))
+
+
+def moe_ep_layout(shape, ep: moe_ep, win: moe_ep_windows, stream=None) -> None:
+    _check("moe_ep_layout", lib().moe_ep_layout(ctypes.byref(shape), ctypes.byref(ep), ctypes.byref(win),
+                                                _stream(stream)))
+
+
+def moe_ep_dispatch(shape, ep: moe_ep, x, topk_idx, win: moe_ep_windows, pos, stream=None) -> None:
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(ctypes.byref(shape), ctypes.byref(ep), _ptr(x),
+                                                    _ptr(topk_idx), ctypes.byref(win), _ptr(pos),
+                                                    _stream(stream)))
+
+
+def moe_ep_grouped_ffn(shape, ep: moe_ep, w: moe_weights, win: moe_ep_windows, stream=None) -> None:
+    _check("moe_ep_grouped_ffn", lib().moe_ep_grouped_ffn(ctypes.byref(shape), ctypes.byref(ep), ctypes.byref(w),
+                                                          ctypes.byref(win), _stream(stream)))
+
+
+def moe_ep_combine(shape, ep: moe_ep, pos, topk_w, win: moe_ep_windows, out, stream=None) -> None:
+    _check("moe_ep_combine", lib().moe_ep_combine(ctypes.byref(shape), ctypes.byref(ep), _ptr(pos), _ptr(topk_w),
+                                                  ctypes.byref(win), _ptr(out), _stream(stream)))
 
 
 def moe_pack_mx_scales(src: torch.Tensor, stream=None) -> torch.Tensor:

@@ -403,6 +403,111 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_shape* shape, const void* x, c
 MOE_API moe_status moe_pack_mx_scales(int64_t n, int64_t rows, int64_t cols, const void* src, void* dst,
                                       moe_stream_t stream);
 
+/* ---- expert parallelism ------------------------------------------------------
+ *
+ * R ranks (one per GPU of one NVLink domain) each own E / R experts, rank d
+ * experts [d E/R, (d + 1) E/R), and each dispatches its own tokens. The pages'
+ * design (NVLinkOneSided abstract): every source rank pushes its tokens,
+ * without exchanging metadata first, into rank-major buffers on the target
+ * ranks, where the grouped GEMM reads them in place; Fence and Sentinel are
+ * the two ways to synchronise, for throughput and for latency.
+ *
+ * Windows. Every rank receives into the windows of V = E virtual experts,
+ * v = el * R + src for local expert el and source rank src: the rows one
+ * source sends one expert form that source's own region, so it fills it with
+ * its own counters and nobody else's.
+ *   MOE_EP_SENTINEL  regions of round_up(t_max, 128) rows; a source publishes
+ *                    each filled 128-row tile with a sentinel word and, when
+ *                    done, its partial tiles and its per-region counts; the
+ *                    receiver's grouped FFN starts once all R sources closed
+ *   MOE_EP_FENCE     sources first write their per-expert pair counts to the
+ *                    owners (moe_ep_count), each owner lays its regions out
+ *                    back to back in whole tiles (moe_ep_layout), and sources
+ *                    then place rows at exact offsets: smaller windows
+ *                    (prefill), one more round of flags
+ * Tokens, h and y keep the single-GPU formats (moe_dispatch_bufs).
+ *
+ * Addressing. Rank d's windows and workspace are reached at d * stride inside
+ * rank-major address ranges that cover all ranks (moe_ep_windows): one
+ * allocation when the ranks are emulated on one device, or, across GPUs, each
+ * peer's allocation mapped into consecutive parts of one reserved virtual
+ * range (CUDA virtual memory management with imported peer handles). Every
+ * cross-rank write is a plain store or atomic to peer memory over NVLink,
+ * released at system scope; no TMA multicast and no library kernel ever
+ * reads a peer's memory, and the grouped FFN reads only its own rank's part.
+ *
+ * Per layer, every rank enqueues, in order: moe_route (with the global
+ * shape), [Fence: moe_ep_count, then moe_ep_layout], moe_ep_dispatch,
+ * moe_ep_grouped_ffn, moe_ep_combine. Cross-rank waits inside those calls are
+ * bounded (MOE_ERR_TIMEOUT after 200 ms). Ranks emulated on one device must
+ * enqueue each step for every rank before the next step of any rank (stream
+ * order then satisfies every wait before it starts).
+ */
+enum { MOE_EP_SENTINEL = 0, MOE_EP_FENCE = 1 };
+
+typedef struct moe_ep {
+  int32_t ranks;      /* R, 1..64, dividing E */
+  int32_t rank;       /* this rank, 0..R-1 */
+  int32_t protocol;   /* MOE_EP_SENTINEL or MOE_EP_FENCE */
+  int32_t reserved;   /* 0 */
+  int64_t t_max;      /* most tokens any rank dispatches in one call (shape->T <= t_max) */
+} moe_ep;
+
+/* Rank-major address ranges: rank d's part starts at d * rows rows (or at
+ * d * ws_bytes bytes for ws), rows and ws_bytes from moe_ep_sizes. */
+typedef struct moe_ep_windows {
+  void* xq;          /* [R * rows, H] xq_dtype: tokens pushed by the sources */
+  float* xs;         /* [R * rows, H/128] fp32 scales (e4m3 tokens, else NULL) */
+  int32_t* row_src;  /* [R * rows]: src * t_max * topk + (t * topk + j) of each placed row */
+  void* hq;          /* [R * rows, I] h_dtype: written by each owner in its own part */
+  float* hs;         /* [R * rows, I/128] (e4m3 h, else NULL) */
+  void* y;           /* [R * rows, H] y_dtype: each owner's expert outputs */
+  void* ws;          /* [R * ws_bytes]: each rank's workspace (moe_ep_workspace_init) */
+} moe_ep_windows;
+
+/* Rows of one rank's windows and bytes of one rank's workspace (host only).
+ * `shape` is the global layer (E = all experts, T = this rank's tokens). */
+MOE_API moe_status moe_ep_sizes(const moe_shape* shape, const moe_ep* ep, int64_t* rows, size_t* ws_bytes);
+
+/* Prepare this rank's workspace (its part of all->ws): counters zeroed, epoch 1. */
+MOE_API moe_status moe_ep_workspace_init(const moe_shape* shape, const moe_ep* ep,
+                                         const moe_ep_windows* all, moe_stream_t stream);
+
+/* Fence, first step: this rank's pair counts per expert, written to the
+ * owners' workspaces (topk_idx [T, topk] from moe_route). */
+MOE_API moe_status moe_ep_count(const moe_shape* shape, const moe_ep* ep, const int32_t* topk_idx,
+                                const moe_ep_windows* all, moe_stream_t stream);
+
+/* Fence, second step: once all R sources' counts are here, lay this rank's
+ * regions out (whole tiles, back to back) and flag the layout ready. */
+MOE_API moe_status moe_ep_layout(const moe_shape* shape, const moe_ep* ep, const moe_ep_windows* all,
+                                 moe_stream_t stream);
+
+/* Push this rank's tokens into their owners' windows (one-pass: atomic claim
+ * in the source's own region, e4m3 per-128 quantisation as moe_dispatch,
+ * sentinel per filled tile, partial tiles and counts at close).
+ *   x   [T, H] act_dtype; topk_idx [T, topk] (global experts)
+ *   pos [T * topk] int32 (out): d * rows + r for a pair placed in row r of
+ *       rank d's windows, -1 if not placed (MOE_ERR_CAPACITY latched) */
+MOE_API moe_status moe_ep_dispatch(const moe_shape* shape, const moe_ep* ep, const void* x,
+                                   const int32_t* topk_idx, const moe_ep_windows* all, int32_t* pos,
+                                   moe_stream_t stream);
+
+/* This rank's grouped FFN over the rows all sources pushed into its windows
+ * (waits, bounded, until all R sources have closed), then its y flagged ready.
+ *   w  this rank's E/R experts' weights, laid out as moe_weights for E/R experts */
+MOE_API moe_status moe_ep_grouped_ffn(const moe_shape* shape, const moe_ep* ep, const moe_weights* w,
+                                      const moe_ep_windows* all, moe_stream_t stream);
+
+/* Weighted combine of this rank's tokens, reading every pair's expert output
+ * in place in its owner's window (the Ascend report's relay-free combine):
+ * out[t] = sum_j topk_w[t, j] * y_all[pos[t * topk + j]], as moe_combine
+ * (identity experts read the pushed tokens). Waits, bounded, until every
+ * owner has flagged its y ready. */
+MOE_API moe_status moe_ep_combine(const moe_shape* shape, const moe_ep* ep, const int32_t* pos,
+                                  const float* topk_w, const moe_ep_windows* all, void* out,
+                                  moe_stream_t stream);
+
 /*
  * Synchronises `stream`, returns the first device error latched in `ws`
  * since the last poll (MOE_OK if none) and clears it.
