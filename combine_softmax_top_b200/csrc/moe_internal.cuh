@@ -337,6 +337,9 @@ cudaError_t launch_ffn_simt(const Ctx& c, const moe_dispatch_bufs& b, const moe_
 cudaError_t launch_ffn_tc(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w,
                           void* y);
 bool ffn_tc_supported(const moe_shape& s);
+// The CTA-pair grouped FFN (e4m3 weights, many rows per expert).
+bool ffn_pair_supported(const Ctx& c);
+cudaError_t launch_ffn_pair(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y);
 
 // expert parallelism (ep.cu); g describes this rank, `all` the rank-major ranges
 cudaError_t launch_ep_count(const Ctx& c, const EpGeom& g, const int32_t* idx, const moe_ep_windows& all);
