@@ -55,9 +55,11 @@ constexpr int kPOffSfa = kPOffB + kPBRows * kSlab;
 constexpr int kPOffSfb = kPOffSfa + kSfAtomBytes;
 constexpr int kPStride = (kPOffSfb + 3 * kSfAtomBytes + 1023) / 1024 * 1024;
 // control: barriers | job queue | flags | reductions | token max exchange |
-// inverse scales | SwiGLU swap buffers
+// inverse scales | SwiGLU swap buffers | weight scale atoms of two jobs
 constexpr int kPSwapBytes = 2 * 2 * 2 * 16 * 32 * 4;   // [set][feature half][direction][16 columns][32 lanes]
-constexpr int kPCtlBytes = 9216 + kPSwapBytes;
+constexpr int kPMaxGroups = 16;                         // K groups of four 128-value blocks (K <= 8192)
+constexpr int kPTabBytes = 2 * kPMaxGroups * 128;       // [job parity][group][8 rows x 16 B]
+constexpr int kPCtlBytes = 9216 + kPSwapBytes + kPTabBytes;
 constexpr int kPStages = (kMaxDynSmem - kPCtlBytes - kTileTabBytes - 1024) / kPStride;
 constexpr int kPSmemBytes = kPStages * kPStride + kPCtlBytes + kTileTabBytes + 1024;
 static_assert(kPStages >= 4 && kPStages <= 8, "pipeline depth");
@@ -140,14 +142,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
   uint8_t* ctl = smem + kPStages * kPStride;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctl);   // [kPStages] even CTA: both halves landed
   uint64_t* empty = full + kPStages;                   // [kPStages] each CTA: the stage's MMAs are done
-  uint64_t* sfa_ready = empty + kPStages;              // [kPStages] even CTA: the odd CTA wrote its scale atom
-  uint64_t* acc_full = sfa_ready + kPStages;           // each CTA: the job's accumulators are complete
+  uint64_t* acc_full = empty + kPStages;               // each CTA: the job's accumulators are complete
   uint64_t* acc_empty = acc_full + 1;                  // even CTA: both epilogues drained them
   uint64_t* drain = acc_empty + 1;
   uint64_t* xchg = drain + 1;                          // [2] each CTA: the peer's token maxima are here
   uint64_t* uq_full = xchg + 2;                        // [kUQ]
   uint64_t* uq_empty = uq_full + kUQ;                  // [kUQ] even CTA: all five consumers took the job
-  static_assert((3 * kPStages + 5 + 2 * kUQ) * 8 <= 512, "barriers fit");
+  uint64_t* tab_free = uq_empty + kUQ;                 // [2] even CTA: a job's scale-atom copies are done
+  static_assert((2 * kPStages + 7 + 2 * kUQ) * 8 <= 512, "barriers fit");
   int4* uq = reinterpret_cast<int4*>(ctl + 512);       // [kUQ]
   int4* epi_job = reinterpret_cast<int4*>(ctl + 640);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 656);
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
   float* amax_peer = reinterpret_cast<float*>(ctl + 4608);    // [2][kPMaxN] written by the peer
   float* sinv = reinterpret_cast<float*>(ctl + 7168);         // [kPMaxN] 1 / scale per token
   float* swap = reinterpret_cast<float*>(ctl + 9216);         // SwiGLU swap buffers
+  uint8_t* sfa_tab = ctl + 9216 + kPSwapBytes;                 // [2][kPMaxGroups][128 B]
   static_assert(7168 + kPMaxN * 4 <= 9216, "control bytes");
 
   const int warp = threadIdx.x >> 5;
@@ -169,7 +172,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
     for (int s = 0; s < kPStages; ++s) {
       ptx::mbar_init(full + s, 1);        // the even CTA's arm, expecting the bytes of both halves
       ptx::mbar_init(empty + s, 1);
-      ptx::mbar_init(sfa_ready + s, 1);
     }
     ptx::mbar_init(acc_full, 1);
     ptx::mbar_init(acc_empty, 2);
@@ -180,6 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       ptx::mbar_init(uq_full + q, 1);
       ptx::mbar_init(uq_empty + q, 5);   // producer, MMA issuer, epilogue (even) + producer, epilogue (odd)
     }
+    ptx::mbar_init(tab_free, 1);
+    ptx::mbar_init(tab_free + 1, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -363,14 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       const int nsteps = down ? p.nk2 : p.nk1;
       const int we = j.e / p.R;
       const int nkb = down ? p.I / 128 : p.H / 128;
-      // this CTA's weight rows, and the exponents of their block scales: lane
-      // l holds blocks l and l + 32 (gate / down in sa, up in sb)
+      // this CTA's weight rows; the even CTA writes the scale atoms of both
+      // (gate/up: the same slice, so the same atom; down: slices 2 p and
+      // 2 p + 1), whose exponents lane l holds for blocks l and l + 32 (gate
+      // or slice 2 p in sa, up or slice 2 p + 1 in sb)
       const int slice_w = down ? 2 * j.slice + (int)rank : j.slice;
-      const float* pa = down ? p.sd + ((int64_t)we * p.n_hslices + slice_w) * nkb
-                             : p.sg + ((int64_t)we * p.n_islices + slice_w) * nkb;
-      const float* pb = down ? pa : p.su + ((int64_t)we * p.n_islices + slice_w) * nkb;
+      const float* pa = down ? p.sd + ((int64_t)we * p.n_hslices + 2 * j.slice) * nkb
+                             : p.sg + ((int64_t)we * p.n_islices + j.slice) * nkb;
+      const float* pb = down ? pa + nkb : p.su + ((int64_t)we * p.n_islices + j.slice) * nkb;
       uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
-      int sbase = 0;
+      const int sbase = 0;   // K <= 8192: every block's exponent is held from the start
       auto load_scales = [&](int b0) {
         bool bad = false;
         auto take = [&](const float* src, int kb) -> uint32_t {
@@ -393,7 +399,35 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         }
         return w;
       };
-      load_scales(0);
+      // the job's weight scale atoms, once (the even CTA, for both): group g
+      // of four K blocks is 8 identical 16-byte rows (the copy reads them
+      // with a zero stride between its four 8-row core matrices). Row m of
+      // A is lane m % 32, column m / 32 of an atom: gate/up rows 0-63 are
+      // gate and 64-127 up, so columns 0-1 hold the gate exponents and 2-3
+      // the up ones. The table of this job's parity is rewritten only after
+      // the copies of the job two before it are done.
+      if (rank == 0) {
+        const uint32_t tp = i & 1u;
+        int t_ok = 1;
+        if (i >= 2 && lane == 0)
+          t_ok = wait_bar(tab_free + tp, ((i >> 1) - 1u) & 1u, abort_flag, hdr, 0x43000000u | tp);
+        if (!__shfl_sync(0xffffffffu, t_ok, 0)) break;
+        load_scales(0);
+        const int ngroups = (nkb + 3) / 4;
+        uint8_t* tab = sfa_tab + tp * (kPMaxGroups * 128);
+        for (int g = 0; g < ngroups; ++g) {
+          const uint32_t wa = pack4(sa0, sa1, 4 * g);
+          const uint32_t wb = pack4(sb0, sb1, 4 * g);
+          const uint4 own = down ? make_uint4(wa, wa, wa, wa) : make_uint4(wa, wa, wb, wb);
+          const uint4 odd = down ? make_uint4(wb, wb, wb, wb) : own;
+          if (lane < 8) reinterpret_cast<uint4*>(tab + g * 128)[lane] = own;
+          else if (lane < 16)
+            ptx::st_cluster_v4(remote(tab + g * 128, 1) + (uint32_t)(lane - 8) * 16u,
+                               make_int4((int)odd.x, (int)odd.y, (int)odd.z, (int)odd.w));
+        }
+        ptx::fence_proxy_async_cluster();   // both tables -> the pair's copies
+        __syncwarp();
+      }
       const int arow_g = we * p.I + j.slice * 128 + 64 * (int)rank;    // gate/up: this CTA's 64 features
       const int arow_d = we * p.H + slice_w * 128;                       // down: this CTA's slice
       const int brow = j.slot * kTileRows;
@@ -409,19 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         uint8_t* st = smem + stage * kPStride;
         const int kb0 = st_i;   // one 128-value K block per stage
         const bool sf_stage = (kb0 & 3) == 0;
-        if (sf_stage) {
-          // weight scale atom: row m of A in lane m % 32, column m / 32; gate/up
-          // rows 0-63 are gate and 64-127 up, so columns 0-1 hold the gate
-          // exponents and 2-3 the up ones
-          if (kb0 + 3 >= sbase + 64) {
-            sbase = kb0;
-            load_scales(sbase);
-          }
-          const uint32_t wa = pack4(sa0, sa1, kb0 - sbase);
-          const uint32_t wb = pack4(sb0, sb1, kb0 - sbase);
-          reinterpret_cast<uint4*>(st + kPOffSfa)[lane] = down ? make_uint4(wa, wa, wa, wa) : make_uint4(wa, wa, wb, wb);
-          ptx::fence_proxy_async_smem();
-        }
         __syncwarp();
         if (ptx::elect_one()) {
           const uint32_t tx = (uint32_t)(kABytes + (h1 + h2) * kSlab + (sf_stage ? j.ntl * kSfAtomBytes : 0));
@@ -442,9 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
               ptx::tma_load_2d_pair(st + kPOffSfb + t * kSfAtomBytes, tmsf, fb, 0,
                                     (j.slot + t) * groups + kb0 / 4);
           }
-          // the odd CTA's scale atom (generic writes, read by the pair's
-          // tcgen05.cp) is published at cluster scope, on the stages that have one
-          if (rank == 1 && sf_stage) ptx::mbar_arrive_cluster(remote(sfa_ready + stage, 0));
         }
         __syncwarp();
         if (rank == 0) {
@@ -469,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (even CTA)
     if (rank == 0) {
-      uint32_t stage = 0, phase = 0, acc_ph = 0, sfa_ph = 0;
+      uint32_t stage = 0, phase = 0, acc_ph = 0;
       for (uint32_t i = 0;; ++i) {
         int4 raw = make_int4(0, 0, kKindAbort << 12, 0);
         if (lane == 0) {
@@ -492,12 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         for (int st_i = 0; st_i < nsteps; ++st_i) {
           int w_ok = 1;
           const int kb0 = st_i;
-          if (lane == 0) {
-            w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x61000000u | stage);
-            if (w_ok && (kb0 & 3) == 0)
-              w_ok = wait_bar<true>(sfa_ready + stage, (sfa_ph >> stage) & 1u, abort_flag, hdr, 0x62000000u | stage);
-          }
-          if ((kb0 & 3) == 0) sfa_ph ^= 1u << stage;
+          if (lane == 0) w_ok = wait_bar(full + stage, phase, abort_flag, hdr, 0x61000000u | stage);
           if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = 0; break; }
           ptx::tc_fence_after();
           uint8_t* st = smem + stage * kPStride;
@@ -507,7 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
                 ptx::tmem_cp_32x128b_x4_pair(tmem + col,
                                              ptx::smem_desc(ptx::smem_u32(st + off), 16, 128, ptx::kLayoutNone));
               };
-              sf_cp(kPColSfa, kPOffSfa);
+              const uint8_t* ta = sfa_tab + ((i & 1u) * kPMaxGroups + kb0 / 4) * 128;
+              ptx::tmem_cp_32x128b_x4_pair(tmem + kPColSfa,
+                                           ptx::smem_desc(ptx::smem_u32(ta), 16, 0, ptx::kLayoutNone));
               for (int t = 0; t < j.ntl; ++t) sf_cp(kPColSfb + 4 * t, kPOffSfb + t * kSfAtomBytes);
             }
             const uint32_t id = (uint32_t)(kb0 & 3);
@@ -537,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         if (ptx::elect_one()) {
           ptx::mma_commit_pair(remote(acc_full, 0));
           ptx::mma_commit_pair(remote(acc_full, 1));
+          ptx::mma_commit_pair(remote(tab_free + (i & 1u), 0));   // this job's scale-atom table is free
         }
         __syncwarp();
         acc_ph ^= 1u;
@@ -748,7 +764,7 @@ bool ffn_pair_supported(const Ctx& c) {
   const moe_shape& s = c.s;
   return s.weight_dtype == MOE_E4M3 && s.xq_dtype == MOE_E4M3 && s.h_dtype == MOE_E4M3 &&
          s.y_dtype == MOE_BF16 && !s.identity_experts && (s.H / 128) % 2 == 0 && s.H % 128 == 0 &&
-         s.I % 128 == 0 && c.s.E <= 1024;
+         s.I % 128 == 0 && s.H <= 128 * 4 * kPMaxGroups && s.I <= 128 * 4 * kPMaxGroups && c.s.E <= 1024;
 }
 
 cudaError_t launch_ffn_pair(const Ctx& c, const moe_dispatch_bufs& b, const moe_weights& w, void* y) {

@@ -54,6 +54,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// generic-proxy writes to the shared memory of any CTA of the cluster ->
+// visible to the async proxy (a pair's tcgen05.cp reading the other CTA)
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
 // generic-proxy writes to global memory (other CTAs, after an acquire) -> async proxy
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
