@@ -821,7 +821,8 @@ cudaError_t launch_ffn_pair(const Ctx& c, const moe_dispatch_bufs& b, const moe_
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(2 * (c.num_sms / 2)), 1, 1);
+  const int pairs = std::max(1, c.num_sms / 2);   // at least one pair, even on a one-SM share
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kPSmemBytes;
   cfg.stream = c.stream;
@@ -829,8 +830,8 @@ cudaError_t launch_ffn_pair(const Ctx& c, const moe_dispatch_bufs& b, const moe_
   cfg.numAttrs = 1;
   int clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&clusters, ffn_pair_kernel<0>, &cfg) == cudaSuccess && clusters > 0)
-    cfg.gridDim.x = (unsigned)(2 * std::min(clusters, c.num_sms / 2));
-  if (cfg.gridDim.x < 2) cfg.gridDim.x = 2;
+    cfg.gridDim.x = (unsigned)(2 * std::min(clusters, pairs));
+  (void)cudaGetLastError();   // a failed query is not the launch's error
   return cudaLaunchKernelEx(&cfg, ffn_pair_kernel<0>, p);
 }
 
