@@ -249,16 +249,18 @@ def ffn_flops(spec, rows):
 TRAFFIC_JSON = os.path.join(PROFILES, "traffic.json")
 
 
-def recorded_traffic(kernel_tag: str):
-    """DRAM bytes per launch of the FFN kernel for one workload, from the
-    record `python bench.py --record-traffic` wrote from an ncu capture, if
-    that capture was taken on the current source of the kernel (else None)."""
+def recorded_traffic(kernel_tag: str, algorithmic_bytes: int):
+    """DRAM bytes per launch of the FFN kernel for one workload: the ratio of
+    DRAM bytes to algorithmic bytes that `python bench.py --record-traffic`
+    took from an ncu capture of a smaller case of the same kernel variant,
+    applied to this launch's algorithmic bytes; None unless the capture was
+    taken on the current source of the kernel."""
     if not os.path.exists(TRAFFIC_JSON):
         return None
     rec = json.load(open(TRAFFIC_JSON)).get(kernel_tag)
-    if not rec or rec.get("source_sha") != kernel_source_sha():
+    if not rec or rec.get("source_sha") != kernel_source_sha() or "traffic_ratio" not in rec:
         return None
-    return int(rec["dram_bytes_per_launch"])
+    return int(round(rec["traffic_ratio"] * algorithmic_bytes))
 
 
 def ncu_dram_bytes(csv_path: str, kernel_regex: str):
@@ -286,11 +288,26 @@ def ncu_dram_bytes(csv_path: str, kernel_regex: str):
 
 
 def record_traffic(args):
-    """Write one profiles/traffic.json entry from an ncu capture."""
+    """Write one profiles/traffic.json entry from an ncu capture of the
+    workload named by --config/--T/--E/--compact: its DRAM bytes per launch
+    over the launch's algorithmic bytes (routing recomputed on the host from
+    the same seeded logits, top-k on the logits)."""
+    import numpy as np
+    import torch
+    from combine_softmax_top_b200 import workloads as W
     mean, n = ncu_dram_bytes(args.record_traffic, args.kernel)
+    spec = W.spec(args.config, **overrides(args))
+    inp = W.make_inputs(spec, seed=args.seed, device="cpu", with_weights=False)
+    idx = torch.topk(inp["logits"], spec.k, dim=1).indices
+    counts = torch.bincount(idx.flatten(), minlength=spec.E).numpy()
+    if spec.shared:
+        counts = np.concatenate([counts, [spec.T]])
+    algo, touched = ffn_algorithmic_bytes(spec, counts)
     rec = json.load(open(TRAFFIC_JSON)) if os.path.exists(TRAFFIC_JSON) else {}
-    rec[args.tag] = {"source_sha": kernel_source_sha(), "dram_bytes_per_launch": int(round(mean)),
-                     "launches": n, "kernel": args.kernel, "how": args.how}
+    rec[args.tag] = {"source_sha": kernel_source_sha(), "traffic_ratio": mean / algo,
+                     "captured": {"workload": workload_config(spec, 1)["workload"], "dram_bytes_per_launch": int(round(mean)),
+                                  "algorithmic_bytes_per_launch": int(algo), "touched_experts": touched, "launches": n},
+                     "kernel": args.kernel, "how": args.how}
     with open(TRAFFIC_JSON, "w") as f:
         json.dump(rec, f, indent=1, sort_keys=True)
         f.write("\n")
@@ -803,7 +820,8 @@ def measure_extras(args, dec_inp, dev, stream, flush, world):
             "l2": "flushed (256 MB write) before every timed step",
             "clocks": clk,
         }
-        out[key]["roofline"]["traffic"] = recorded_traffic(f"grouped_ffn/{spec.name}")
+        out[key]["roofline"]["traffic"] = recorded_traffic(f"grouped_ffn/{spec.name}",
+                                                           out[key]["roofline"]["algorithmic_bytes_per_launch"])
         if key == "prefill":
             out[key]["overlap"] = time_overlap(spec, inp, dev, flush, args.steps, args.warmup)
         del inp, b
@@ -920,7 +938,8 @@ def run_ours(args):
                     "algorithmic_bytes_per_launch": both["algorithmic_bytes_per_launch"],
                     "flops_per_launch": both["flops_per_launch"], "touched_experts": both["touched_experts"],
                     "launch_ms": ffn_ms, "peak_source": top["peak_how"],
-                    "traffic": recorded_traffic(f"grouped_ffn/{spec.name}")}
+                    "traffic": recorded_traffic(f"grouped_ffn/{spec.name}",
+                                                both["algorithmic_bytes_per_launch"])}
 
     extras = {}
     if args.config == "decode" and not overrides(args) and not args.no_extra:
