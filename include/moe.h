@@ -10,7 +10,10 @@
  *   moe_grouped_ffn  every expert's SwiGLU FFN over its rows, read in place
  *   moe_combine      top-k weighted gather-reduce back to token order
  *
- * and moe_layer, which enqueues all four. The stage split follows the pages:
+ * and moe_layer, which enqueues all four; moe_layer_overlap, the same layer with
+ * dispatch running beside the grouped FFN on a partition of the SMs; and the
+ * expert-parallel calls moe_ep_* (experts split over ranks, tokens pushed into
+ * the owners' rank-major windows). The stage split follows the pages:
  * an MoE layer is token dispatch, grouped GEMMs and a combine (GC-MoE feed
  * item, "Key points"; GC-MoE explainer, "Why Expert Parallelism Is
  * Inefficient in MoE Decoding"); dispatch pushes tokens into per-expert
