@@ -55,10 +55,11 @@ constexpr int kPOffSfa = kPOffB + kPBRows * kSlab;
 constexpr int kPOffSfb = kPOffSfa + kSfAtomBytes;
 constexpr int kPStride = (kPOffSfb + 3 * kSfAtomBytes + 1023) / 1024 * 1024;
 // control: barriers | job queue | flags | reductions | token max exchange |
-// inverse scales | SwiGLU swap buffers | weight scale atoms of two jobs
+// inverse scales | SwiGLU swap buffers | weight scale atoms of three jobs
 constexpr int kPSwapBytes = 2 * 2 * 2 * 16 * 32 * 4;   // [set][feature half][direction][16 columns][32 lanes]
 constexpr int kPMaxGroups = 16;                         // K groups of four 128-value blocks (K <= 8192)
-constexpr int kPTabBytes = 2 * kPMaxGroups * 128;       // [job parity][group][8 rows x 16 B]
+constexpr int kPTabRing = 3;                            // scale-atom tables in flight (built ahead by the scheduler)
+constexpr int kPTabBytes = kPTabRing * kPMaxGroups * 128;   // [job % 3][group][8 rows x 16 B]
 constexpr int kPCtlBytes = 9216 + kPSwapBytes + kPTabBytes;
 constexpr int kPStages = (kMaxDynSmem - kPCtlBytes - kTileTabBytes - 1024) / kPStride;
 constexpr int kPSmemBytes = kPStages * kPStride + kPCtlBytes + kTileTabBytes + 1024;
@@ -148,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
   uint64_t* xchg = drain + 1;                          // [2] each CTA: the peer's token maxima are here
   uint64_t* uq_full = xchg + 2;                        // [kUQ]
   uint64_t* uq_empty = uq_full + kUQ;                  // [kUQ] even CTA: all five consumers took the job
-  uint64_t* tab_free = uq_empty + kUQ;                 // [2] even CTA: a job's scale-atom copies are done
-  static_assert((2 * kPStages + 7 + 2 * kUQ) * 8 <= 512, "barriers fit");
+  uint64_t* tab_free = uq_empty + kUQ;                 // [3] even CTA: a job's scale-atom copies are done
+  static_assert((2 * kPStages + 5 + kPTabRing + 2 * kUQ) * 8 <= 512, "barriers fit");
   int4* uq = reinterpret_cast<int4*>(ctl + 512);       // [kUQ]
   int4* epi_job = reinterpret_cast<int4*>(ctl + 640);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 656);
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
   float* amax_peer = reinterpret_cast<float*>(ctl + 4608);    // [2][kPMaxN] written by the peer
   float* sinv = reinterpret_cast<float*>(ctl + 7168);         // [kPMaxN] 1 / scale per token
   float* swap = reinterpret_cast<float*>(ctl + 9216);         // SwiGLU swap buffers
-  uint8_t* sfa_tab = ctl + 9216 + kPSwapBytes;                 // [2][kPMaxGroups][128 B]
+  uint8_t* sfa_tab = ctl + 9216 + kPSwapBytes;                 // [kPTabRing][kPMaxGroups][128 B]
   static_assert(7168 + kPMaxN * 4 <= 9216, "control bytes");
 
   const int warp = threadIdx.x >> 5;
@@ -182,8 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       ptx::mbar_init(uq_full + q, 1);
       ptx::mbar_init(uq_empty + q, 5);   // producer, MMA issuer, epilogue (even) + producer, epilogue (odd)
     }
-    ptx::mbar_init(tab_free, 1);
-    ptx::mbar_init(tab_free + 1, 1);
+    for (int t = 0; t < kPTabRing; ++t) ptx::mbar_init(tab_free + t, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -267,71 +267,150 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         __syncwarp();
       }
       const uint32_t ntiles = p.streaming ? 0u : ld_acquire(misc + kRingTotal);
-      if (lane == 0) {
-        uint32_t i = 0;
-        bool good = !*abort_flag;
-        auto push = [&](const PJob& j) -> bool {
-          const uint32_t q = i % kUQ, ph = (i / kUQ) & 1u;
-          if (!wait_bar<true>(uq_empty + q, ph ^ 1u, abort_flag, hdr, 0x91000000u | q)) return false;
-          const int4 v = pack(j);
-          uq[q] = v;
-          ptx::st_cluster_v4(remote(uq + q, 1), v);
-          ptx::mbar_arrive(uq_full + q);
-          ptx::mbar_arrive_cluster(remote(uq_full + q, 1));
-          ++i;
-          return true;
+      uint32_t i = 0;   // jobs pushed so far (the queue index; every lane keeps it)
+      auto push = [&](const PJob& j) -> bool {   // lane 0
+        const uint32_t q = i % kUQ, ph = (i / kUQ) & 1u;
+        if (!wait_bar<true>(uq_empty + q, ph ^ 1u, abort_flag, hdr, 0x91000000u | q)) return false;
+        const int4 v = pack(j);
+        uq[q] = v;
+        ptx::st_cluster_v4(remote(uq + q, 1), v);
+        ptx::mbar_arrive(uq_full + q);
+        ptx::mbar_arrive_cluster(remote(uq_full + q, 1));
+        return true;
+      };
+      // The weight scale atoms of job i, for both CTAs (warp-wide): e4m3
+      // weights have one scale per 128 x 128 block, so an atom's 32 rows are
+      // identical and a K group of four blocks is 8 rows of 16 bytes (the
+      // copy reads them with a zero stride between its four 8-row core
+      // matrices). Row m of A is lane m % 32, column m / 32 of an atom:
+      // gate/up rows 0-63 are gate and 64-127 up (columns 0-1 gate, 2-3 up);
+      // a down job's even CTA holds slice 2 p, the odd one 2 p + 1. Built a
+      // few jobs ahead in a ring of three tables, each rewritten only after
+      // the copies of the job three before it are done, so that neither the
+      // loads nor the MMAs wait for it.
+      auto build_table = [&](const PJob& j) -> bool {
+        const bool down = j.kind == kKindDown;
+        const int we = j.e / p.R;
+        const int nkb = down ? p.I / 128 : p.H / 128;
+        const float* pa = down ? p.sd + ((int64_t)we * p.n_hslices + 2 * j.slice) * nkb
+                               : p.sg + ((int64_t)we * p.n_islices + j.slice) * nkb;
+        const float* pb = down ? pa + nkb : p.su + ((int64_t)we * p.n_islices + j.slice) * nkb;
+        const uint32_t ts = i % kPTabRing;
+        int t_ok = 1;
+        if (i >= (uint32_t)kPTabRing && lane == 0)
+          t_ok = wait_bar(tab_free + ts, (i / kPTabRing - 1u) & 1u, abort_flag, hdr, 0x43000000u | ts);
+        if (!__shfl_sync(0xffffffffu, t_ok, 0)) return false;
+        bool bad = false;
+        auto take = [&](const float* src, int kb) -> uint32_t {
+          const float v = __ldg(src + kb);
+          bad |= !pow2_scale_ok(v);
+          return ue8m0(v);
         };
-        if (good && !p.streaming && (uint32_t)ntab != ntiles) {
+        uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;   // exponents of blocks lane and lane + 32
+        if (lane < nkb) { sa0 = take(pa, lane); sb0 = take(pb, lane); }
+        if (lane + 32 < nkb) { sa1 = take(pa, lane + 32); sb1 = take(pb, lane + 32); }
+        if (__ballot_sync(0xffffffffu, bad) != 0u && lane == 0)
+          latch_error(hdr, MOE_ERR_INVALID_ARG, 0x25000000u | (uint32_t)we);
+        auto pack4 = [&](uint32_t r0, uint32_t r1, int kr) -> uint32_t {
+          uint32_t w = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int kk = kr + b;
+            const uint32_t v = __shfl_sync(0xffffffffu, kk < 32 ? r0 : r1, kk & 31);
+            w |= (kk < nkb ? v : 0u) << (8 * b);
+          }
+          return w;
+        };
+        uint8_t* tab = sfa_tab + ts * (kPMaxGroups * 128);
+        for (int g = 0; g < (nkb + 3) / 4; ++g) {
+          const uint32_t wa = pack4(sa0, sa1, 4 * g);
+          const uint32_t wb = pack4(sb0, sb1, 4 * g);
+          const uint4 own = down ? make_uint4(wa, wa, wa, wa) : make_uint4(wa, wa, wb, wb);
+          const uint4 odd = down ? make_uint4(wb, wb, wb, wb) : own;
+          if (lane < 8) reinterpret_cast<uint4*>(tab + g * 128)[lane] = own;
+          else if (lane < 16)
+            ptx::st_cluster_v4(remote(tab + g * 128, 1) + (uint32_t)(lane - 8) * 16u,
+                               make_int4((int)odd.x, (int)odd.y, (int)odd.z, (int)odd.w));
+        }
+        ptx::fence_proxy_async_cluster();   // both tables -> the pair's copies
+        __syncwarp();
+        return true;
+      };
+      bool good = !*abort_flag;
+      {
+        int ok = 1;
+        if (lane == 0 && good && !p.streaming && (uint32_t)ntab != ntiles) {
           latch_error(hdr, MOE_ERR_INVALID_ARG, 0x24000000u | (uint32_t)ntab);
           *abort_flag = 1;
-          good = false;
+          ok = 0;
         }
-        const uint32_t nchunks = (uint32_t)chunk_tab[p.E];
-        const uint32_t npairs = (uint32_t)(p.n_hslices / 2);
-        const uint32_t n1 = nchunks * (uint32_t)p.n_islices;
-        const uint32_t total = n1 + nchunks * npairs;
-        while (good) {
+        good = good && __shfl_sync(0xffffffffu, ok, 0);
+      }
+      const uint32_t nchunks = (uint32_t)chunk_tab[p.E];
+      const uint32_t npairs = (uint32_t)(p.n_hslices / 2);
+      const uint32_t n1 = nchunks * (uint32_t)p.n_islices;
+      const uint32_t total = n1 + nchunks * npairs;
+      while (good) {
+        // lane 0 resolves the next unit (1: a job, 0: none left, -1: a wait failed)
+        int state = 0;
+        int4 jv = make_int4(0, 0, 0, 0);
+        if (lane == 0) {
           const uint32_t u = atomicAdd(misc + kFfnNext, 1u);
-          if (u >= total) break;
-          PJob j;
-          j.kind = u >= n1 ? kKindDown : kKindGateUp;
-          const uint32_t v = j.kind == kKindDown ? u - n1 : u;
-          const uint32_t ns = j.kind == kKindDown ? npairs : (uint32_t)p.n_islices;
-          // weight expert (R windows each, expert parallelism), then slice-major
-          const int R = p.R;
-          int lo = 0, hi = p.E / R - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((uint32_t)chunk_tab[mid * R] * ns <= v) lo = mid;
-            else hi = mid - 1;
-          }
-          const int c0 = chunk_tab[lo * R];
-          const uint32_t nc = (uint32_t)(chunk_tab[(lo + 1) * R] - c0);
-          const uint32_t w = v - (uint32_t)c0 * ns;
-          const int cc = c0 + (int)(w % nc);
-          int ve = lo * R;
-          while (ve + 1 < (lo + 1) * R && chunk_tab[ve + 1] <= cc) ++ve;
-          j.e = ve;
-          j.slice = (int)(w / nc);
-          const int ci = cc - chunk_tab[ve];                       // chunk within the window
-          const int nchv = chunk_tab[ve + 1] - chunk_tab[ve];
-          const int c = (int)min(ld_acquire(cnt + ve), (uint32_t)p.cap);
-          const int nt = (c + kTileRows - 1) / kTileRows;
-          j.ntl = ci == nchv - 1 ? nt - 2 * ci : 2;
-          j.slot = (base ? (int)base[ve] : ve * p.tpe) + 2 * ci;
-          int rows = 0;
-          for (int t = 0; good && t < j.ntl; ++t) {
-            int r = 0;
-            good = wait_tile(p.ws, epoch, j.slot + t, abort_flag, &r);
-            rows += r;
-          }
-          if (!good) break;
-          j.rows = rows;
-          if (j.kind == kKindDown)   // both CTAs of every gate/up job of this chunk stored their h
-            good = wait_count(hdone + j.slot, 2u * (uint32_t)p.n_islices * (gen + 1u), abort_flag, hdr,
+          if (u < total) {
+            PJob j;
+            j.kind = u >= n1 ? kKindDown : kKindGateUp;
+            const uint32_t v = j.kind == kKindDown ? u - n1 : u;
+            const uint32_t ns = j.kind == kKindDown ? npairs : (uint32_t)p.n_islices;
+            // weight expert (R windows each, expert parallelism), then slice-major
+            const int R = p.R;
+            int lo = 0, hi = p.E / R - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if ((uint32_t)chunk_tab[mid * R] * ns <= v) lo = mid;
+              else hi = mid - 1;
+            }
+            const int c0 = chunk_tab[lo * R];
+            const uint32_t nc = (uint32_t)(chunk_tab[(lo + 1) * R] - c0);
+            const uint32_t w = v - (uint32_t)c0 * ns;
+            const int cc = c0 + (int)(w % nc);
+            int ve = lo * R;
+            while (ve + 1 < (lo + 1) * R && chunk_tab[ve + 1] <= cc) ++ve;
+            j.e = ve;
+            j.slice = (int)(w / nc);
+            const int ci = cc - chunk_tab[ve];                       // chunk within the window
+            const int nchv = chunk_tab[ve + 1] - chunk_tab[ve];
+            const int c = (int)min(ld_acquire(cnt + ve), (uint32_t)p.cap);
+            const int nt = (c + kTileRows - 1) / kTileRows;
+            j.ntl = ci == nchv - 1 ? nt - 2 * ci : 2;
+            j.slot = (base ? (int)base[ve] : ve * p.tpe) + 2 * ci;
+            bool ok = true;
+            int rows = 0;
+            for (int t = 0; ok && t < j.ntl; ++t) {
+              int r = 0;
+              ok = wait_tile(p.ws, epoch, j.slot + t, abort_flag, &r);
+              rows += r;
+            }
+            j.rows = rows;
+            if (ok && j.kind == kKindDown)   // both CTAs of every gate/up job of this chunk stored their h
+              ok = wait_count(hdone + j.slot, 2u * (uint32_t)p.n_islices * (gen + 1u), abort_flag, hdr,
                               0x31000000u | (uint32_t)j.slot);
-          if (good) good = push(j);
+            state = ok ? 1 : -1;
+            jv = pack(j);
+          }
         }
+        state = __shfl_sync(0xffffffffu, state, 0);
+        if (state <= 0) {
+          good = state == 0;
+          break;
+        }
+        const PJob j = unpack(shfl_int4(jv));
+        if (!build_table(j)) { good = false; break; }
+        int pok = 1;
+        if (lane == 0) pok = push(j);
+        if (!__shfl_sync(0xffffffffu, pok, 0)) { good = false; break; }
+        ++i;
+      }
+      if (lane == 0) {
         PJob end;
         end.e = end.slice = end.rows = end.ntl = end.slot = 0;
         end.kind = good ? kKindEnd : kKindAbort;
@@ -367,67 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       const int nsteps = down ? p.nk2 : p.nk1;
       const int we = j.e / p.R;
       const int nkb = down ? p.I / 128 : p.H / 128;
-      // this CTA's weight rows; the even CTA writes the scale atoms of both
-      // (gate/up: the same slice, so the same atom; down: slices 2 p and
-      // 2 p + 1), whose exponents lane l holds for blocks l and l + 32 (gate
-      // or slice 2 p in sa, up or slice 2 p + 1 in sb)
-      const int slice_w = down ? 2 * j.slice + (int)rank : j.slice;
-      const float* pa = down ? p.sd + ((int64_t)we * p.n_hslices + 2 * j.slice) * nkb
-                             : p.sg + ((int64_t)we * p.n_islices + j.slice) * nkb;
-      const float* pb = down ? pa + nkb : p.su + ((int64_t)we * p.n_islices + j.slice) * nkb;
-      uint32_t sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
-      const int sbase = 0;   // K <= 8192: every block's exponent is held from the start
-      auto load_scales = [&](int b0) {
-        bool bad = false;
-        auto take = [&](const float* src, int kb) -> uint32_t {
-          const float v = __ldg(src + kb);
-          bad |= !pow2_scale_ok(v);
-          return ue8m0(v);
-        };
-        if (lane + b0 < nkb) { sa0 = take(pa, b0 + lane); sb0 = take(pb, b0 + lane); }
-        if (lane + b0 + 32 < nkb) { sa1 = take(pa, b0 + lane + 32); sb1 = take(pb, b0 + lane + 32); }
-        if (__ballot_sync(0xffffffffu, bad) != 0u && lane == 0)
-          latch_error(hdr, MOE_ERR_INVALID_ARG, 0x25000000u | (uint32_t)we);
-      };
-      auto pack4 = [&](uint32_t r0, uint32_t r1, int kr) -> uint32_t {
-        uint32_t w = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int kk = kr + b;
-          const uint32_t v = __shfl_sync(0xffffffffu, kk < 32 ? r0 : r1, kk & 31);
-          w |= (kk + sbase < nkb ? v : 0u) << (8 * b);
-        }
-        return w;
-      };
-      // the job's weight scale atoms, once (the even CTA, for both): group g
-      // of four K blocks is 8 identical 16-byte rows (the copy reads them
-      // with a zero stride between its four 8-row core matrices). Row m of
-      // A is lane m % 32, column m / 32 of an atom: gate/up rows 0-63 are
-      // gate and 64-127 up, so columns 0-1 hold the gate exponents and 2-3
-      // the up ones. The table of this job's parity is rewritten only after
-      // the copies of the job two before it are done.
-      if (rank == 0) {
-        const uint32_t tp = i & 1u;
-        int t_ok = 1;
-        if (i >= 2 && lane == 0)
-          t_ok = wait_bar(tab_free + tp, ((i >> 1) - 1u) & 1u, abort_flag, hdr, 0x43000000u | tp);
-        if (!__shfl_sync(0xffffffffu, t_ok, 0)) break;
-        load_scales(0);
-        const int ngroups = (nkb + 3) / 4;
-        uint8_t* tab = sfa_tab + tp * (kPMaxGroups * 128);
-        for (int g = 0; g < ngroups; ++g) {
-          const uint32_t wa = pack4(sa0, sa1, 4 * g);
-          const uint32_t wb = pack4(sb0, sb1, 4 * g);
-          const uint4 own = down ? make_uint4(wa, wa, wa, wa) : make_uint4(wa, wa, wb, wb);
-          const uint4 odd = down ? make_uint4(wb, wb, wb, wb) : own;
-          if (lane < 8) reinterpret_cast<uint4*>(tab + g * 128)[lane] = own;
-          else if (lane < 16)
-            ptx::st_cluster_v4(remote(tab + g * 128, 1) + (uint32_t)(lane - 8) * 16u,
-                               make_int4((int)odd.x, (int)odd.y, (int)odd.z, (int)odd.w));
-        }
-        ptx::fence_proxy_async_cluster();   // both tables -> the pair's copies
-        __syncwarp();
-      }
+      const int slice_w = down ? 2 * j.slice + (int)rank : j.slice;   // down: this CTA's slice of H
       const int arow_g = we * p.I + j.slice * 128 + 64 * (int)rank;    // gate/up: this CTA's 64 features
       const int arow_d = we * p.H + slice_w * 128;                       // down: this CTA's slice
       const int brow = j.slot * kTileRows;
@@ -520,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
                 ptx::tmem_cp_32x128b_x4_pair(tmem + col,
                                              ptx::smem_desc(ptx::smem_u32(st + off), 16, 128, ptx::kLayoutNone));
               };
-              const uint8_t* ta = sfa_tab + ((i & 1u) * kPMaxGroups + kb0 / 4) * 128;
+              const uint8_t* ta = sfa_tab + ((i % kPTabRing) * kPMaxGroups + kb0 / 4) * 128;
               ptx::tmem_cp_32x128b_x4_pair(tmem + kPColSfa,
                                            ptx::smem_desc(ptx::smem_u32(ta), 16, 0, ptx::kLayoutNone));
               for (int t = 0; t < j.ntl; ++t) sf_cp(kPColSfb + 4 * t, kPOffSfb + t * kSfAtomBytes);
@@ -552,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         if (ptx::elect_one()) {
           ptx::mma_commit_pair(remote(acc_full, 0));
           ptx::mma_commit_pair(remote(acc_full, 1));
-          ptx::mma_commit_pair(remote(tab_free + (i & 1u), 0));   // this job's scale-atom table is free
+          ptx::mma_commit_pair(remote(tab_free + i % kPTabRing, 0));   // this job's scale-atom table is free
         }
         __syncwarp();
         acc_ph ^= 1u;
