@@ -589,8 +589,9 @@ def time_overlap(spec, inp, dev, flush, steps, warmup, splits=(8, 20, 32), green
     gives dispatch P SMs' worth of CTAs and the FFN's persistent grid the
     other SMs; it is timed stream-launched and as the replay of a CUDA graph
     of one call (route and the counting pass, then dispatch and the FFN as
-    two concurrent branches, then combine). `green` splits put the dispatch
-    stream in a green context of P SMs instead."""
+    two concurrent branches, then combine). `green` splits enforce the
+    partition with two green contexts (P SMs for dispatch, the rest for the
+    layer's other kernels), stream-launched only."""
     import numpy as np
     import torch
     from combine_softmax_top_b200 import moe
@@ -643,14 +644,19 @@ def time_overlap(spec, inp, dev, flush, steps, warmup, splits=(8, 20, 32), green
             continue
 
         def over(ov=ov):
-            moe.moe_layer_overlap(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, ov.ov)
+            moe.overlap_layer(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, ov)
 
         try:
-            r = {"us": timed(over) * 1e3, "graph_us": graphed(over) * 1e3}
+            r = {"us": timed(over) * 1e3}
+            if is_green:
+                r["dispatch_sms"], r["main_sms"] = ov.ov.dispatch_sms, ov.ov.ffn_sms
+            else:
+                r["graph_us"] = graphed(over) * 1e3
         except Exception as exc:
             r = {"unavailable": str(exc)[:200]}
         else:
             r["same_bits"] = bool(torch.equal(lw.out, ref))
+        ov.close()
         res["splits"][key] = r
     best = min((v["us"], k) for k, v in res["splits"].items() if "us" in v)
     res["best"] = {"split": best[1], "us": best[0], "gain_vs_serial": res["serial_us"] / best[0]}

@@ -387,15 +387,73 @@ def run_layer_ws(lw: LayerWorkspace, inp: dict, stream=None) -> None:
     moe_layer(lw.shape, inp["x"], inp["logits"], w, lw.ws, lw.out, stream)
 
 
+class GreenPartition:
+    """Two green contexts over disjoint SM sets of one device, one stream
+    each: `dispatch_sms` SMs (rounded up by the driver to its split
+    granularity) for dispatch, every other SM for the rest of the layer.
+    Both sides must be confined: a kernel on an ordinary stream may run on
+    any SM, so a persistent grouped FFN there can take the SMs of a
+    dispatch-only green context and leave dispatch none, and the FFN's
+    tile waits then run out. Made with the driver's SM-resource split
+    (cuda.bindings); released by close()."""
+
+    def __init__(self, dispatch_sms: int, index: int):
+        from cuda.bindings import driver as cu
+        self._cu = cu
+        self._ctxs, self._streams = [], []
+
+        def call(fn, *args):
+            r = fn(*args)
+            if r[0] != cu.CUresult.CUDA_SUCCESS:
+                raise RuntimeError(f"{fn.__name__} failed: {r[0]}")
+            return r[1] if len(r) == 2 else r[1:]
+
+        try:
+            call(cu.cuInit, 0)
+            dev = call(cu.cuDeviceGet, index)
+            sm = call(cu.cuDeviceGetDevResource, dev, cu.CUdevResourceType.CU_DEV_RESOURCE_TYPE_SM)
+            groups, n, rest = call(cu.cuDevSmResourceSplitByCount, 1, sm, 0, int(dispatch_sms))
+            if n < 1 or groups[0].sm.smCount < 1 or rest.sm.smCount < 1:
+                raise RuntimeError(f"no SM split of {dispatch_sms} on device {index}")
+            # dispatch: high priority, it is the producer the grouped FFN waits on
+            for res, prio in ((groups[0], -1), (rest, 0)):
+                desc = call(cu.cuDevResourceGenerateDesc, [res], 1)
+                g = call(cu.cuGreenCtxCreate, desc, dev, cu.CUgreenCtxCreate_flags.CU_GREEN_CTX_DEFAULT_STREAM)
+                self._ctxs.append(g)
+                self._streams.append(call(cu.cuGreenCtxStreamCreate, g, cu.CUstream_flags.CU_STREAM_NON_BLOCKING,
+                                          prio))
+        except Exception:
+            self.close()
+            raise
+        self.dispatch_sms = int(groups[0].sm.smCount)
+        self.main_sms = int(rest.sm.smCount)
+        self.dispatch_stream = int(self._streams[0])
+        self.main_stream = int(self._streams[1])
+
+    def close(self) -> None:
+        cu = self._cu
+        for st in self._streams:
+            cu.cuStreamSynchronize(st)
+            cu.cuStreamDestroy(st)
+        for g in self._ctxs:
+            cu.cuGreenCtxDestroy(g)
+        self._streams, self._ctxs = [], []
+
+
 class Overlap:
     """A dispatch stream and the fork/join events moe_layer_overlap orders it
-    with (torch objects; the library only borrows their handles). With
-    green=True the dispatch stream belongs to a green context of
-    dispatch_sms SMs (torch.cuda.GreenContext), so the partition is enforced
-    by the device; otherwise the grouped FFN's grid leaves those SMs free."""
+    with (torch objects; the library only borrows their handles). Without
+    green, the grouped FFN's persistent grid leaves dispatch_sms SMs free and
+    dispatch runs on a second stream of the caller's context. With
+    green=True the device enforces the split: dispatch runs on a green
+    context of dispatch_sms SMs and the layer itself (route, counting pass,
+    grouped FFN, combine) on a green context of all the other SMs
+    (GreenPartition); `main` is that stream, and overlap_layer orders it
+    after and before the caller's stream."""
 
     def __init__(self, dispatch_sms: int, ffn_sms: int = 0, green: bool = False, device=None):
-        self.green_ctx = None
+        self.partition = None
+        self.main = None
         if device is None:
             index = torch.cuda.current_device()
         elif isinstance(device, int):
@@ -403,9 +461,11 @@ class Overlap:
         else:
             index = torch.device(device).index or 0
         if green:
-            self.green_ctx = torch.cuda.GreenContext.create(int(dispatch_sms), int(index))
-            self._green_stream = self.green_ctx.Stream()
-            self.stream = torch.cuda.ExternalStream(self._green_stream.native_handle)
+            self.partition = GreenPartition(dispatch_sms, index)
+            self.stream = torch.cuda.ExternalStream(self.partition.dispatch_stream, device=index)
+            self.main = torch.cuda.ExternalStream(self.partition.main_stream, device=index)
+            dispatch_sms = self.partition.dispatch_sms
+            ffn_sms = min(ffn_sms, self.partition.main_sms) if ffn_sms else self.partition.main_sms
         else:
             # a high-priority stream: dispatch is the producer the FFN waits on
             # (and high-priority streams never double as graph-capture streams)
@@ -423,10 +483,29 @@ class Overlap:
         self.ov.dispatch_sms = dispatch_sms
         self.ov.ffn_sms = ffn_sms
 
+    def close(self) -> None:
+        if self.partition is not None:
+            torch.cuda.synchronize()
+            self.partition.close()
+            self.partition = None
+
+
+def overlap_layer(shape, x, logits, w: moe_weights, ws, out, ov: Overlap, stream=None) -> None:
+    """moe_layer_overlap on `stream`, or, for a green split, on its main
+    stream ordered after the caller's stream and before whatever the caller
+    enqueues next."""
+    if ov.main is None:
+        moe_layer_overlap(shape, x, logits, w, ws, out, ov.ov, stream)
+        return
+    cur = torch.cuda.current_stream() if stream is None else stream
+    ov.main.wait_stream(cur)
+    moe_layer_overlap(shape, x, logits, w, ws, out, ov.ov, ov.main)
+    cur.wait_stream(ov.main)
+
 
 def run_layer_overlap(lw: "LayerWorkspace", inp: dict, ov: Overlap, stream=None) -> None:
     """Enqueue one whole layer with dispatch beside the grouped FFN."""
-    moe_layer_overlap(lw.shape, inp["x"], inp["logits"], weights_struct(inp), lw.ws, lw.out, ov.ov, stream)
+    overlap_layer(lw.shape, inp["x"], inp["logits"], weights_struct(inp), lw.ws, lw.out, ov, stream)
 
 
 # kernels the library launches per stage (mirrors the launch plan in csrc/)

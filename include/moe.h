@@ -318,9 +318,16 @@ MOE_API moe_status moe_layer_bufs(const moe_shape* shape, const void* x, const f
  * How moe_layer_overlap splits the device between dispatch and the grouped
  * FFN (all caller-owned; the library creates no stream or event).
  *   dispatch_stream  a second stream, not the legacy default stream, that
- *                    the dispatch kernel runs on; with a green context of
- *                    dispatch_sms SMs (torch.cuda.GreenContext) its SMs are
- *                    the partition's, else the SMs the grouped FFN leaves
+ *                    the dispatch kernel runs on. On two streams of one
+ *                    context the split is by grid size: the grouped FFN's
+ *                    persistent CTAs hold ffn_sms SMs and dispatch takes the
+ *                    SMs they leave. For a split the device enforces, both
+ *                    `stream` and dispatch_stream must belong to green
+ *                    contexts over disjoint SM sets (ffn_sms at most the
+ *                    former's SMs): a green context for dispatch alone does
+ *                    not confine the FFN, whose CTAs may then occupy every
+ *                    SM of dispatch's partition, so that its tile waits run
+ *                    out (MOE_ERR_TIMEOUT)
  *   fork_event       cudaEvent_t (cudaEventDisableTiming is enough):
  *   join_event       recorded on `stream` / dispatch_stream to order the two
  *   dispatch_sms     SMs dispatch is sized for: its grid is one wave of

@@ -73,16 +73,24 @@ def test_overlap_matches_serial_layer_and_oracle(name, base, over, dsms, cuda_de
     assert err < TOL[s.weight], err
 
 
+@pytest.mark.parametrize("green", [False, True], ids=["stream", "green"])
 @pytest.mark.parametrize("name,over", [
     ("decode", {}),                       # the full decode layer (e4m3, 11 GB of weights)
     ("prefill", dict(compact=1)),         # the full prefill layer on compact windows
 ])
-def test_overlap_full_size_bitwise(name, over, cuda_device):
+def test_overlap_full_size_bitwise(name, over, green, cuda_device):
+    """Full layers, the split left to the FFN's grid size or enforced by two
+    green contexts (a persistent FFN beside a dispatch-only green context
+    could take dispatch's SMs; both sides confined, it cannot)."""
+    if green:
+        pytest.importorskip("cuda.bindings.driver")
     torch.cuda.empty_cache()
     s = W.spec(name, **over)
     inp = W.make_inputs(s, seed=0, device="cuda")
     ref = _serial(s, inp)
-    (out,) = _overlapped(s, inp, moe.Overlap(20))
+    ov = moe.Overlap(20, green=green)
+    (out,) = _overlapped(s, inp, ov)
+    ov.close()
     assert torch.equal(out, ref)
     # a token sample against the oracle
     idx, _ = oracle.route(raw(inp["logits"]), s.k, s.renorm)
@@ -109,17 +117,21 @@ def test_overlap_partition_sizes(dsms, ffn, cuda_device):
     assert torch.equal(out, ref)
 
 
-def test_overlap_on_a_green_context(cuda_device):
-    """Dispatch on a stream of a green context of 20 SMs, the SM partition
-    enforced by the device (where torch was built with green contexts)."""
-    if not torch.cuda.green_contexts.SUPPORTED:
-        pytest.skip("torch built without green contexts")
+def test_overlap_on_green_contexts(cuda_device):
+    """The partition enforced by the device: dispatch on a green context of
+    20 SMs (rounded up to the driver's split granularity), the rest of the
+    layer on a green context of all the other SMs."""
+    pytest.importorskip("cuda.bindings.driver")
     s = W.spec("decode", T=1024, H=512, E=8, k=2, I=256)
     inp = W.make_inputs(s, seed=4, device="cuda")
     ref = _serial(s, inp)
     ov = moe.Overlap(20, green=True)
-    (out,) = _overlapped(s, inp, ov)
-    assert torch.equal(out, ref)
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    assert 20 <= ov.ov.dispatch_sms and ov.ov.dispatch_sms + ov.ov.ffn_sms <= n
+    outs = _overlapped(s, inp, ov, calls=2)
+    ov.close()
+    for o in outs:
+        assert torch.equal(o, ref)
 
 
 def test_overlap_dispatch_held_back_times_out_cleanly(cuda_device):
