@@ -58,6 +58,10 @@ def parse():
     p.add_argument("--overlap-sweep", action="store_true",
                    help="print one JSON line per workload (decode, prefill on compact windows) timing "
                         "the layer with dispatch beside the grouped FFN over a sweep of partition sizes")
+    p.add_argument("--fp8-gemm-peak", action="store_true",
+                   help="print one JSON line: cuBLAS e4m3 GEMM throughput on this GPU (8192^3, "
+                        "tensor-wise scales), best of 10 and back to back for 4 s with clocks, for "
+                        "context beside the 2 x bf16 roof")
     p.add_argument("--report", action="store_true",
                    help="instead of the single bench line: one JSON line per workload "
                         "(tiny, decode, prefill, skew, dispatch+combine sweep) with per-stage "
@@ -666,6 +670,51 @@ def time_overlap(spec, inp, dev, flush, steps, warmup, splits=(8, 20, 32), green
     return res
 
 
+def run_fp8_gemm_peak(args):
+    """A library e4m3 GEMM (torch._scaled_mm, i.e. cuBLAS) on this GPU: the
+    dense FP8 rate a plain GEMM reaches here, burst (best of 10 launches) and
+    under the power cap (back to back for 4 s, clocks sampled meanwhile).
+    Context for the prefill FFN's tensor fraction, not a roof of its own."""
+    import torch
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    n = 8192
+    a = (torch.randn(n, n, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn)
+    b = (torch.randn(n, n, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device="cuda")
+
+    def mm():
+        return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    clocks = ClockSampler(0)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    calls, t0 = 0, time.time()
+    e0.record()
+    while time.time() - t0 < 4.0:
+        for _ in range(20):
+            mm()
+        calls += 20
+        torch.cuda.synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    print(json.dumps({"metric": "cuBLAS e4m3 GEMM 8192^3", "burst_tflops": flop / (best * 1e-3) / 1e12,
+                      "sustained_tflops": flop * calls / (e0.elapsed_time(e1) * 1e-3) / 1e12,
+                      "clocks": clocks.stop(), "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, tensor-wise scales"}))
+
+
 def run_overlap_sweep(args):
     import torch
     from combine_softmax_top_b200 import workloads as W
@@ -768,10 +817,14 @@ def ffn_roofline(spec, counts, ffn_ms, peaks, peak_kind, burst=True):
     t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (tc_peak * 1e12)
     src = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    # the same roof at the power-capped rate: the FFN is timed inside a loop
+    # of back-to-back layers, where the part runs at its power cap
+    sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (tc_peak / bf16)
     return {"bound": "hbm" if t_hbm >= t_tc else "tensor",
             "tensor": {"achieved": tfs, "peak": tc_peak, "unit": "TFLOP/s", "frac": tfs / tc_peak,
                        "peak_how": ("2 x " if tc_peak != bf16 else "") +
-                                   ("burst" if burst else "sustained") + " bf16 GEMM, " + src},
+                                   ("burst" if burst else "sustained") + " bf16 GEMM, " + src,
+                       "peak_sustained": sus, "frac_sustained": tfs / sus},
             "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                     "peak_how": "copy bandwidth, " + src},
             "algorithmic_bytes_per_launch": abytes, "flops_per_launch": flops, "touched_experts": touched,
@@ -997,6 +1050,8 @@ def main():
         run_report(args)
     elif args.overlap_sweep:
         run_overlap_sweep(args)
+    elif args.fp8_gemm_peak:
+        run_fp8_gemm_peak(args)
     else:
         run_ours(args)
 

@@ -29,13 +29,16 @@
 //            slice 2 p + r of W_down, and its D those 128 features of y.
 // A chunk is two 128-row tiles of one expert, or one; an expert's last tile
 // joins the chunk before it when it holds at most kPTail rows. Its token
-// columns go to two MMAs: N1 <= 256 and, for a joined tile, N2 <= kPTail.
+// columns go to one MMA (N <= 256) or, with a joined tile, to two: the first
+// tile (N1 = 128) and the rest (N2 <= 192).
 //
 // Roles per CTA (352 threads): warp 10 of the even CTA schedules jobs into
 // both CTAs' queues; warp 0 of each CTA loads its half of every stage (the
 // odd CTA's copies complete on the even CTA's barrier, whose expected bytes
 // count both halves); warp 1 of the even CTA issues all MMAs and commits to both
-// CTAs' barriers; warps 2-9 of each CTA drain their own tensor memory. Every
+// CTAs' barriers; warps 2-9 of each CTA drain their own tensor memory,
+// consecutive jobs' accumulators sitting at opposite ends of it so that the
+// next job's MMAs start once the overlapping columns are drained. Every
 // wait is bounded; on expiry the kernel latches MOE_ERR_TIMEOUT, drains,
 // meets its peer at a cluster barrier, frees tensor memory and exits.
 #include "ffn_common.cuh"
@@ -65,8 +68,20 @@ constexpr int kPStages = (kMaxDynSmem - kPCtlBytes - kTileTabBytes - 1024) / kPS
 constexpr int kPSmemBytes = kPStages * kPStride + kPCtlBytes + kTileTabBytes + 1024;
 static_assert(kPStages >= 4 && kPStages <= 8, "pipeline depth");
 static_assert(kPSmemBytes <= kMaxDynSmem, "shared memory");
-constexpr uint32_t kPColSfa = 448, kPColSfb = 452;   // accumulators use columns 0 .. kPMaxN - 1
-static_assert(kPMaxN <= 448, "tensor memory");
+// Tensor memory: the scale factors in the last 16 columns (one weight atom,
+// up to three token atoms), accumulators below them. Consecutive jobs take
+// opposite ends of the accumulator columns: job i from column 0 when i is
+// even, else ending at kPAccEnd (its first column rounded down to 32), so
+// that two jobs of up to kPMaxN columns overlap in at most 160 columns. The
+// epilogue drains the columns the next job will write first and frees the
+// accumulator then; the MMAs of the next job run while it drains the rest.
+constexpr uint32_t kPColSfa = 496, kPColSfb = kPColSfa + 4;
+constexpr int kPAccEnd = (int)kPColSfa;
+constexpr int kPOddMin = (kPAccEnd - kPMaxN) / 32 * 32;   // lowest first column of an odd job
+static_assert(kPColSfb + 12 <= 512 && kPOddMin >= 128, "tensor memory");
+__device__ __forceinline__ int acc_base(uint32_t job, int ncol) {
+  return (job & 1u) ? (kPAccEnd - ncol) / 32 * 32 : 0;
+}
 
 struct PairParams {
   CUtensorMap tm_wg, tm_wu;       // gate / up weights, boxes of 64 rows
@@ -116,10 +131,14 @@ __device__ __forceinline__ int chunks_of(int c) {
   return (nt & 1) && nt >= 3 && last <= kPTail ? nt / 2 : (nt + 1) / 2;
 }
 
-// Token columns of the two MMAs of a job of `rows` rows (multiples of 32, so
-// that each CTA's half is a whole number of 16-row boxes).
+// Token columns of the MMAs of a job of `rows` rows (multiples of 32, so that
+// each CTA's half is a whole number of 16-row boxes): one MMA up to 256, else
+// the first tile (128) and the rest (at most 192). An MMA's time has a floor
+// of about 80 cycles at small N and grows with N above it, so 128 + 192
+// costs less than 256 plus a thin MMA of the joined tile's rows. The second
+// MMA starts on a tile boundary, where its token scales start a scale atom.
 __device__ __forceinline__ void split_n(int rows, int* n1, int* n2) {
-  const int a = min(rows, 256), b = rows - a;
+  const int a = rows > 256 ? 128 : rows, b = rows - a;
   *n1 = (a + 31) & ~31;
   *n2 = b > 0 ? (b + 31) & ~31 : 0;
 }
@@ -476,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
           }
           // token rows: this CTA's half of each MMA's columns
           load_rows(tmt, st + kPOffB, fb, kx, brow + (int)rank * h1, h1);
-          if (h2) load_rows(tmt, st + kPOffB + h1 * kSlab, fb, kx, brow + 256 + (int)rank * h2, h2);
+          if (h2) load_rows(tmt, st + kPOffB + h1 * kSlab, fb, kx, brow + n1 + (int)rank * h2, h2);
           if (sf_stage) {   // the chunk's token scale atoms (the same in both CTAs)
             for (int t = 0; t < j.ntl; ++t)
               ptx::tma_load_2d_pair(st + kPOffSfb + t * kSfAtomBytes, tmsf, fb, 0,
@@ -524,6 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         ptx::tc_fence_after();
         const int nsteps = down ? p.nk2 : p.nk1;
+        const uint32_t d1 = tmem + (uint32_t)acc_base(i, n1 + n2);   // this job's first accumulator column
         const uint32_t idesc1 = ptx::idesc_mxf8(256, n1, 0);
         const uint32_t idesc2 = ptx::idesc_mxf8(256, n2 > 0 ? n2 : 16, 0);
         for (int st_i = 0; st_i < nsteps; ++st_i) {
@@ -550,15 +570,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
             const uint64_t b2 = ptx::desc_kmajor_sw128(st + kPOffB + h1 * kSlab);
             const uint32_t sfa = (tmem + kPColSfa) | (id << 30);
             const uint32_t sfb1 = (tmem + kPColSfb) | (id << 30);
-            const uint32_t sfb2 = (tmem + kPColSfb + 8) | (id << 30);   // the joined tile's atom
+            const uint32_t sfb2 = (tmem + kPColSfb + 4u * (uint32_t)(n1 / 128)) | (id << 30);   // from its first tile's atom
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t off = (uint64_t)(kk * 32) >> 4;
               const uint32_t acc = (st_i > 0 || kk > 0) ? 1u : 0u;
-              ptx::mma_mxf8_pair(tmem, a + off, b1 + off, idesc1 | (id << 4) | (id << 29), sfa, sfb1, acc);
+              ptx::mma_mxf8_pair(d1, a + off, b1 + off, idesc1 | (id << 4) | (id << 29), sfa, sfb1, acc);
               if (n2)
-                ptx::mma_mxf8_pair(tmem + (uint32_t)n1, a + off, b2 + off, idesc2 | (id << 4) | (id << 29), sfa,
-                                   sfb2, acc);
+                ptx::mma_mxf8_pair(d1 + (uint32_t)n1, a + off, b2 + off, idesc2 | (id << 4) | (id << 29), sfa, sfb2,
+                                   acc);
             }
             // the stage is free in both CTAs once these MMAs are done
             ptx::mma_commit_pair(remote(empty + stage, 0));
@@ -623,19 +643,40 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       const bool down = j.kind == kKindDown;
       int n1, n2;
       split_n(j.rows, &n1, &n2);
-      const int ncol = n1 + n2;   // column c holds chunk row c
+      const int ncol = n1 + n2;   // column base + c holds chunk row c
+      const int nb = ncol / 32;     // 32-column batches
       const int64_t row0 = (int64_t)j.slot * kTileRows;
+      // The batches the next job's accumulator overlaps are drained first:
+      // an even job's high ones (the next job starts at kPOddMin or above, so
+      // the drain runs from the last batch down), an odd job's low ones (the
+      // next starts at column 0 and ends below kPMaxN). The accumulator is
+      // freed once each set has drained rel_bi batches.
+      const bool odd = (i & 1u) != 0u;
+      const uint32_t base = (uint32_t)acc_base(i, ncol);
+      const int n_pre = odd ? min(nb, max(0, kPMaxN - (int)base + 31) / 32) : max(0, nb - kPOddMin / 32);
+      const int rel_bi = (n_pre + 1) / 2;
+      auto col_of = [&](int pos) { return 32 * (odd ? pos : nb - 1 - pos); };   // chunk row of a batch
+      auto release = [&]() {   // 2. the overlapped columns are drained in both sets: free them
+        ptx::tc_fence_before();
+        ptx::named_barrier(1, kEpiThreads);
+        if (et == 0) {
+          if (rank == 0) ptx::mbar_arrive(acc_empty);
+          else ptx::mbar_arrive_remote(remote(acc_empty, 0));
+        }
+      };
       // 1. drain into registers: h = SwiGLU (gate/up; this thread's feature,
       //    even columns in the gate warp, odd in the up warp) or y in bf16
       //    pairs (down)
       uint32_t v[kPBatches][16];
 #pragma unroll
       for (int bi = 0; bi < kPBatches; ++bi) {
-        const int c0 = 32 * (eset + 2 * bi);
-        if (c0 >= ncol) break;
+        if (bi == rel_bi) release();
+        const int pos = eset + 2 * bi;
+        if (pos >= nb) continue;   // every thread still reaches the release
+        const int c0 = col_of(pos);
         uint32_t r[32];
-        ptx::tmem_ld_x16(tmem + lane_base + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(r));
-        ptx::tmem_ld_x16(tmem + lane_base + (uint32_t)c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+        ptx::tmem_ld_x16(tmem + lane_base + base + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(r));
+        ptx::tmem_ld_x16(tmem + lane_base + base + (uint32_t)c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
         ptx::tmem_wait_ld();
         if (down) {
 #pragma unroll
@@ -658,21 +699,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
           ptx::named_barrier(pair_bar, 64);   // both read: the buffers are free for the next batch
         }
       }
-      // 2. accumulators drained in both sets: free them for the next job
-      ptx::tc_fence_before();
-      ptx::named_barrier(1, kEpiThreads);
-      if (et == 0) {
-        if (rank == 0) ptx::mbar_arrive(acc_empty);
-        else ptx::mbar_arrive_remote(remote(acc_empty, 0));
-      }
+      if (rel_bi >= kPBatches) release();
       if (down) {
         // 3. y rows: lane = feature of this CTA's slice
         __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(p.y) + row0 * p.H +
                             (2 * j.slice + (int)rank) * 128 + q * 32 + lane;
 #pragma unroll
         for (int bi = 0; bi < kPBatches; ++bi) {
-          const int c0 = 32 * (eset + 2 * bi);
-          if (c0 >= ncol) break;
+          const int pos = eset + 2 * bi;
+          if (pos >= nb) break;
+          const int c0 = col_of(pos);
 #pragma unroll
           for (int k2 = 0; k2 < 16; ++k2) {
             const int c = c0 + 2 * k2;
@@ -689,8 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       const uint32_t apeer_remote = remote(amax_peer + par * kPMaxN, peer);
 #pragma unroll
       for (int bi = 0; bi < kPBatches; ++bi) {
-        const int c0 = 32 * (eset + 2 * bi);
-        if (c0 >= ncol) break;
+        const int pos = eset + 2 * bi;
+        if (pos >= nb) break;
+        const int c0 = col_of(pos);
 #pragma unroll
         for (int k2 = 0; k2 < 16; ++k2) {   // |h| bit patterns order like the values
           const uint32_t m = __reduce_max_sync(0xffffffffu, v[bi][k2] & 0x7FFFFFFFu);
@@ -728,8 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_pair_kernel(const __grid_cons
       uint8_t* hp = reinterpret_cast<uint8_t*>(p.hq) + row0 * p.I + j.slice * 128 + 64 * (int)rank + 32 * fq + lane;
 #pragma unroll
       for (int bi = 0; bi < kPBatches; ++bi) {
-        const int c0 = 32 * (eset + 2 * bi);
-        if (c0 >= ncol) break;
+        const int pos = eset + 2 * bi;
+        if (pos >= nb) break;
+        const int c0 = col_of(pos);
 #pragma unroll
         for (int k2 = 0; k2 < 16; ++k2) {
           const int c = c0 + 2 * k2 + (up_warp ? 1 : 0);
