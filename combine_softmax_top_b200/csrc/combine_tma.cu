@@ -124,21 +124,34 @@ __global__ void __launch_bounds__(threads_of<kRowDt>(), 1) combine_tma_kernel(co
   if (warp == kCompWarps) {
     // ------------------------------------------------------------ loader
     uint32_t armed = 0, armed_parity = 0;
+    // lane j's slot of a unit: its row and weight, loaded one unit ahead so
+    // that the load's latency overlaps the wait for a free stage
+    auto load_meta = [&](int64_t u, int* row, float* wj) {
+      *row = -1;
+      *wj = 0.f;
+      if (u < units && lane < a.k) {
+        const int64_t t = u / a.nparts;
+        *row = __ldg(a.pos + t * a.k + lane);
+        *wj = __ldg(a.w + t * a.k + lane);
+      }
+    };
+    int row_next;
+    float w_next;
+    load_meta(blockIdx.x, &row_next, &w_next);
     for (int i = 0;; ++i) {
       const int64_t u = blockIdx.x + (int64_t)i * gridDim.x;
       if (u >= units) break;
+      const int row = row_next;
+      const float wj = w_next;
+      load_meta(u + gridDim.x, &row_next, &w_next);
       const int s = i % kStages;
       int ok = 1;
       if (lane == 0 && i >= kStages)
         ok = wait_phase(empty + s, ((i / kStages) & 1) ^ 1, &abort_flag, a.hdr, 0xC1000000u | s);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const int t = (int)(u / a.nparts), part = (int)(u % a.nparts);
+      const int part = (int)(u % a.nparts);
       uint8_t* st = smem + s * a.stage_bytes;
-      int row = -1;
-      float wj = 0.f;
       if (lane < a.k) {
-        row = __ldg(a.pos + (int64_t)t * a.k + lane);
-        wj = __ldg(a.w + (int64_t)t * a.k + lane);
         reinterpret_cast<int*>(st + a.off_meta)[lane] = row;
         reinterpret_cast<float*>(st + a.off_meta)[kMaxSlots + lane] = wj;
       }
