@@ -13,8 +13,9 @@
 // row): one loader warp bulk-copies the unit's k row chunks (and, for e4m3
 // identity rows, their scales) into a ring of shared-memory stages, so that
 // two to three units' rows (~115-170 KB) are in flight per SM without
-// holding them in registers; 8 or 16 compute warps read the stage, form the
-// weighted sums 16 values per thread and write the output coalesced. A
+// holding them in registers; 16 compute warps (8 for fp32 rows) read the
+// stage, form the weighted sums over the live slots (compacted by the
+// loader) 8 or 16 values per thread and write the output coalesced. A
 // persistent grid of one CTA per SM walks the units. Every wait is bounded:
 // on expiry the kernel latches MOE_ERR_TIMEOUT, waits (bounded) for its
 // copies and returns.
@@ -24,16 +25,23 @@
 namespace moe {
 namespace {
 
-// compute warps: e4m3 rows carry more arithmetic per byte (decode of each
-// value) and take twice as many; measured, each count is the faster one
+// values per compute thread: one 16-byte shared-memory read per row (8 bf16,
+// 16 e4m3; fp32 rows take four reads of 16 values), so that a warp's reads
+// of a row are consecutive and free of bank conflicts
 template <int kRowDt>
-__host__ __device__ constexpr int comp_warps() { return kRowDt == MOE_E4M3 ? 16 : 8; }
+__host__ __device__ constexpr int vals_of() { return kRowDt == MOE_BF16 ? 8 : 16; }
+// compute warps: 16, so that a unit's groups (V / vals_of) keep 14-16 warps
+// busy; fp32 rows keep 8
+template <int kRowDt>
+__host__ __device__ constexpr int comp_warps() { return kRowDt == MOE_F32 ? 8 : 16; }
 template <int kRowDt>
 __host__ __device__ constexpr int threads_of() { return (comp_warps<kRowDt>() + 1) * 32; }   // + one loader warp
 constexpr int kStages = 3;
 constexpr int kRowCap = 64 * 1024;                // row-chunk bytes of one stage
 constexpr int kMaxSlots = 32;
-constexpr int kMetaBytes = 2 * kMaxSlots * 4;     // pos[32] | w[32]
+// a stage's slot list: the live slots (row copied, weight non-zero) in slot
+// order, compacted by the loader: slot[32] | w[32] | row[32] | count
+constexpr int kMetaBytes = 3 * kMaxSlots * 4 + 16;
 
 struct Args {
   const int32_t* pos;
@@ -50,13 +58,12 @@ struct Args {
 };
 
 template <int kRowDt>
-__device__ __forceinline__ void fma16(const uint8_t* src, float s, float wj, float* acc) {
+__device__ __forceinline__ void fma_vals(const uint8_t* src, float s, float wj, float* acc) {
   if constexpr (kRowDt == MOE_BF16) {
-    const uint4 r0 = reinterpret_cast<const uint4*>(src)[0];
-    const uint4 r1 = reinterpret_cast<const uint4*>(src)[1];
-    const uint32_t u[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    const uint4 r = *reinterpret_cast<const uint4*>(src);
+    const uint32_t u[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
       acc[2 * i] = fmaf(wj, __uint_as_float(u[i] << 16), acc[2 * i]);
       acc[2 * i + 1] = fmaf(wj, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
     }
@@ -151,13 +158,17 @@ __global__ void __launch_bounds__(threads_of<kRowDt>(), 1) combine_tma_kernel(co
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int part = (int)(u % a.nparts);
       uint8_t* st = smem + s * a.stage_bytes;
-      if (lane < a.k) {
-        reinterpret_cast<int*>(st + a.off_meta)[lane] = row;
-        reinterpret_cast<float*>(st + a.off_meta)[kMaxSlots + lane] = wj;
-      }
-      __syncwarp();   // the meta words are written before lane 0's arrive publishes them
       const bool copy = lane < a.k && row >= 0 && wj != 0.f;
-      const uint32_t n = __popc(__ballot_sync(0xffffffffu, copy));
+      const uint32_t live = __ballot_sync(0xffffffffu, copy);
+      const uint32_t n = __popc(live);
+      if (copy) {   // the live slots in slot order, so that the sums keep it
+        const int c = __popc(live & ((1u << lane) - 1u));
+        reinterpret_cast<int*>(st + a.off_meta)[c] = lane;
+        reinterpret_cast<float*>(st + a.off_meta)[kMaxSlots + c] = wj;
+        reinterpret_cast<int*>(st + a.off_meta)[2 * kMaxSlots + c] = row;
+      }
+      if (lane == 0) reinterpret_cast<int*>(st + a.off_meta)[3 * kMaxSlots] = (int)n;
+      __syncwarp();   // the slot list is written before lane 0's arrive publishes it
       const uint32_t bytes = n * (uint32_t)(chunk_bytes + (a.scale_bulk ? nscales * 4 : 0));
       if (lane == 0) ptx::mbar_arrive_expect_tx(full + s, bytes);   // also publishes the meta words
       __syncwarp();
@@ -186,7 +197,8 @@ __global__ void __launch_bounds__(threads_of<kRowDt>(), 1) combine_tma_kernel(co
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute
-    const int ngroups = a.V / 16;
+    constexpr int kVals = vals_of<kRowDt>();
+    const int ngroups = a.V / kVals;
     for (int i = 0;; ++i) {
       const int64_t u = blockIdx.x + (int64_t)i * gridDim.x;
       if (u >= units) break;
@@ -196,39 +208,41 @@ __global__ void __launch_bounds__(threads_of<kRowDt>(), 1) combine_tma_kernel(co
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int t = (int)(u / a.nparts), part = (int)(u % a.nparts);
       const uint8_t* st = smem + s * a.stage_bytes;
-      const int* spos = reinterpret_cast<const int*>(st + a.off_meta);
+      const int* sslot = reinterpret_cast<const int*>(st + a.off_meta);
       const float* sw = reinterpret_cast<const float*>(st + a.off_meta) + kMaxSlots;
+      const int* srow = reinterpret_cast<const int*>(st + a.off_meta) + 2 * kMaxSlots;
+      const int nlive = sslot[3 * kMaxSlots];
       for (int g = threadIdx.x; g < ngroups; g += kCompWarps * 32) {
-        float acc[16];
+        float acc[kVals];
 #pragma unroll
-        for (int v = 0; v < 16; ++v) acc[v] = 0.f;
-        for (int j = 0; j < a.k; ++j) {
-          const int row = spos[j];
-          const float wj = sw[j];
-          if (row < 0 || wj == 0.f) continue;
+        for (int v = 0; v < kVals; ++v) acc[v] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < nlive; ++c) {
+          const int j = sslot[c];
+          const float wj = sw[c];
           float sc = 0.f;
           if constexpr (kRowDt == MOE_E4M3) {
-            const int blk = (g * 16) / kQBlock;
+            const int blk = (g * kVals) / kQBlock;
             sc = a.scale_bulk ? reinterpret_cast<const float*>(st + a.off_scale)[j * nscales + blk]
-                              : __ldg(a.xs + (int64_t)row * (a.H / kQBlock) + (int64_t)part * nscales + blk);
+                              : __ldg(a.xs + (int64_t)srow[c] * (a.H / kQBlock) + (int64_t)part * nscales + blk);
           }
-          fma16<kRowDt>(st + j * chunk_bytes + g * 16 * a.elt, sc, wj, acc);
+          fma_vals<kRowDt>(st + j * chunk_bytes + g * kVals * a.elt, sc, wj, acc);
         }
-        const int64_t off = (int64_t)t * a.H + (int64_t)part * a.V + g * 16;
+        const int64_t off = (int64_t)t * a.H + (int64_t)part * a.V + g * kVals;
         if constexpr (kOutDt == MOE_BF16) {
-          uint32_t wv[8];
+          uint32_t wv[kVals / 2];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < kVals / 2; ++v) {
             __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * v], acc[2 * v + 1]);
             wv[v] = *reinterpret_cast<uint32_t*>(&b2);
           }
           uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + off);
-          p[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          p[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+#pragma unroll
+          for (int v = 0; v < kVals / 8; ++v) p[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
         } else {
           float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + off);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) p[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+          for (int v = 0; v < kVals / 4; ++v) p[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
         }
       }
       __syncwarp();
@@ -286,7 +300,8 @@ bool launch_combine_tma(const Ctx& c, const moe_dispatch_bufs& b, const void* y,
   const int smem = kStages * a.stage_bytes + 128;
   const int grid = (int)std::min<int64_t>((int64_t)T * nparts, c.num_sms);
   const bool bf16_out = c.s.out_dtype == MOE_BF16;
-  const int threads = row_dt == MOE_E4M3 ? threads_of<MOE_E4M3>() : threads_of<MOE_BF16>();
+  const int threads = row_dt == MOE_E4M3 ? threads_of<MOE_E4M3>()
+                      : row_dt == MOE_BF16 ? threads_of<MOE_BF16>() : threads_of<MOE_F32>();
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess) {
