@@ -75,3 +75,40 @@ def test_reference_arm_other_ranks_exit_quietly():
                    {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_ffn_roofline_arithmetic():
+    """The FFN's two roofs: bytes at the copy rate and FLOPs at the tensor
+    rate of its operand type (twice bf16 for 8-bit and 4-bit weights), the
+    higher roof naming the bound, and the same achieved rate against the
+    power-capped (sustained) figure."""
+    import numpy as np
+    from combine_softmax_top_b200 import workloads as W
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200.0}
+    spec = W.spec("prefill")
+    counts = np.full(spec.E, spec.T * spec.k // spec.E, dtype=np.int64)
+    flops = bench.ffn_flops(spec, int(counts.sum()))
+    assert flops == 6.0 * spec.H * spec.I * spec.T * spec.k
+    ms = 3.0
+    r = bench.ffn_roofline(spec, counts, ms, peaks, "measured")
+    t = r["tensor"]
+    assert t["peak"] == 3000.0 and t["peak_sustained"] == 2400.0
+    assert t["achieved"] == pytest.approx(flops / 3e-3 / 1e12)
+    assert t["frac"] == pytest.approx(t["achieved"] / 3000.0)
+    assert t["frac_sustained"] == pytest.approx(t["achieved"] / 2400.0)
+    abytes, touched = bench.ffn_algorithmic_bytes(spec, counts)
+    assert touched == spec.E and r["hbm"]["achieved"] == pytest.approx(abytes / 3e-3 / 1e9)
+    # 256 rows per expert: 5.77 TFLOP against 13 GB (weights, rows, h twice,
+    # y): 1.92 ms at 3 PFLOP/s, 2.16 ms at 6 TB/s, so the byte roof is higher
+    t_tc, t_hbm = flops / 3000e12, abytes / 6000e9
+    assert t_hbm > t_tc and r["bound"] == "hbm"
+    assert bench.ffn_roofline(spec, counts, ms, dict(peaks, hbm_gbs=8000.0), "measured")["bound"] == "tensor"
+    dec = W.spec("decode")
+    dcounts = np.zeros(dec.E, dtype=np.int64)
+    dcounts[: dec.T * dec.k // 4] = 4
+    rd = bench.ffn_roofline(dec, dcounts, 1.7, peaks, "measured")
+    assert rd["bound"] == "hbm"                       # 4 rows per expert: weight streaming
+    assert rd["tensor"]["peak"] == 3000.0             # e4m3 weights: twice bf16
+    bf = W.spec("skew")
+    rb = bench.ffn_roofline(bf, np.full(bf.E, bf.T * bf.k // bf.E), 1.0, peaks, "measured")
+    assert rb["tensor"]["peak"] == 1500.0 and rb["tensor"]["peak_sustained"] == 1200.0
