@@ -112,3 +112,47 @@ def test_ffn_roofline_arithmetic():
     bf = W.spec("skew")
     rb = bench.ffn_roofline(bf, np.full(bf.E, bf.T * bf.k // bf.E), 1.0, peaks, "measured")
     assert rb["tensor"]["peak"] == 1500.0 and rb["tensor"]["peak_sustained"] == 1200.0
+
+
+def test_ncu_dram_bytes_per_launch(tmp_path):
+    """DRAM bytes per launch from an ncu --csv metrics log: read + write per
+    launch ID, units scaled, other kernels and metrics ignored, the banner
+    lines before the header skipped."""
+    cols = ["ID", "Process ID", "Process Name", "Host Name", "Kernel Name", "Context", "Stream",
+            "Block Size", "Grid Size", "Device", "CC", "Section Name", "Metric Name", "Metric Unit",
+            "Metric Value"]
+
+    def row(i, kern, metric, unit, value):
+        return [str(i), "1", "python3", "host", kern, "1", "7", "(352, 1, 1)", "(148, 1, 1)", "0", "10.0",
+                "Command line profiler metrics", metric, unit, value]
+
+    rows = [row(0, "void ffn_tc_kernel<1, 16>(TcParams)", "dram__bytes_read.sum", "Gbyte", "1.5"),
+            row(0, "void ffn_tc_kernel<1, 16>(TcParams)", "dram__bytes_write.sum", "Mbyte", "100"),
+            row(0, "void ffn_tc_kernel<1, 16>(TcParams)", "gpu__time_duration.sum", "us", "900"),
+            row(1, "void combine_kernel<1, 1>(Args)", "dram__bytes_read.sum", "Gbyte", "9"),
+            row(2, "void ffn_tc_kernel<1, 16>(TcParams)", "dram__bytes_read.sum", "byte", "1,300,000,000"),
+            row(2, "void ffn_tc_kernel<1, 16>(TcParams)", "dram__bytes_write.sum", "Kbyte", "100000")]
+    p = tmp_path / "launches.csv"
+    with open(p, "w") as f:
+        f.write("==PROF== Connected to process 1\n")
+        for r in [cols] + rows:
+            f.write(",".join(f'"{c}"' for c in r) + "\n")
+    mean, n = bench.ncu_dram_bytes(str(p), "ffn_tc_kernel")
+    assert n == 2
+    assert mean == pytest.approx((1.5e9 + 100e6 + 1.3e9 + 100e6) / 2)
+    with pytest.raises(ValueError):
+        bench.ncu_dram_bytes(str(p), "ffn_pair")
+
+
+def test_recorded_traffic_only_for_the_current_source(tmp_path, monkeypatch):
+    """A recorded DRAM/algorithmic ratio is applied to a launch's algorithmic
+    bytes only while the FFN sources hash as they did at capture."""
+    rec = {"grouped_ffn/decode": {"source_sha": "abc", "traffic_ratio": 1.01}}
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(p))
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "abc")
+    assert bench.recorded_traffic("grouped_ffn/decode", 1_000_000) == 1_010_000
+    assert bench.recorded_traffic("grouped_ffn/prefill", 1_000_000) is None
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "changed")
+    assert bench.recorded_traffic("grouped_ffn/decode", 1_000_000) is None
